@@ -1,0 +1,370 @@
+/*
+ * hlta_oracle.c -- plain fp64 CPU oracle of the Hybrid Linear Temporal
+ * Attention forward pass (Kairos, arXiv 2606.16533, section 2.2).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file: only the tests, the package's smoke check and the benchmark's CPU
+ * baseline do.  It shares no code with the CUDA library.
+ *
+ * Everything is computed in double precision.  Inputs arrive either as float32
+ * arrays or as bf16 bit patterns (uint16); both hold exact values that are
+ * widened to double before use.
+ *
+ * Layouts (row-major):
+ *   q, k : [B, L, H, d_k]      v, out : [B, L, H, d_v]
+ *   alpha, beta : [B, L, H] float32
+ *   S : [B, H, d_v, d_k] double (S maps keys to values: v ~ S k)
+ *
+ * Functions and the passages they follow:
+ *   oracle_attention  -- section 2.2.2, Eq. (7) (SWA) and Eq. (8) (DSWA), with
+ *                        the causal window and residue-class dilation readings
+ *                        documented beside each predicate below.
+ *   oracle_gdn        -- section 2.2.1, steps 2-4 (Eq. (2)-(6)) and the output
+ *                        o_t = S_t q_t.
+ *   oracle_gdn_chunked-- the same recurrence regrouped into chunks (a
+ *                        derivation from Eq. (6), not on the pages); used only to
+ *                        show that the chunk form computes the recurrence.
+ *
+ * Parity pins for every function live in tests/test_oracle.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* dtype codes of input tensors */
+#define ORC_F32 0
+#define ORC_BF16 1
+
+static inline double load_elem(const void *p, int dt, size_t i) {
+    if (dt == ORC_BF16) {
+        uint32_t u = ((uint32_t)((const uint16_t *)p)[i]) << 16;
+        float f;
+        memcpy(&f, &u, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)p)[i];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention masks (section 2.2.2).                                          */
+/* ------------------------------------------------------------------------ */
+
+/* SWA, Eq. (7), causal reading: query i sees the w most recent keys including
+ * itself, i - w < j <= i.  (The equation prints a centred window; the layer
+ * built here is causal.) */
+static inline int swa_in_window(long i, long j, long w) {
+    return j <= i && j > i - w;
+}
+
+/* DSWA, Eq. (8): SWA applied after rearranging (B, F*P, D) -> (B*d, F/d*P, D).
+ * Reading: frames are split into d residue classes f mod d; within one class
+ * the frames f = g, g+d, g+2d, ... are concatenated in order, so token
+ * t = f*P + s sits at rearranged position r(t) = floor(f/d)*P + s.  Query i
+ * sees key j iff both are in the same class and 0 <= r(i) - r(j) < w. */
+static inline long rearranged_pos(long t, long P, long dil) {
+    long f = t / P, s = t % P;
+    return (f / dil) * P + s;
+}
+
+static inline int dswa_in_window(long i, long j, long P, long dil, long w) {
+    long fi = i / P, fj = j / P;
+    if ((fi - fj) % dil != 0) return 0;
+    long dr = rearranged_pos(i, P, dil) - rearranged_pos(j, P, dil);
+    return dr >= 0 && dr < w;
+}
+
+/*
+ * oracle_attention: softmax attention rows under the SWA (kind 0) or DSWA
+ * (kind 1) mask.
+ *
+ *   logits_j = q_i . k_j / sqrt(d_k) over every key j the mask admits;
+ *   p = softmax(logits) (max-subtracted, fp64 sums);  o_i = sum_j p_j v_j.
+ *
+ * rows: nrows row ids, id = (b*L + t)*H + h, or NULL for all B*L*H rows in
+ * that order.  out: [nrows, d_v] doubles.
+ * span: keys are examined over j in [max(0, i - span), i]; pass span < 0 to
+ * examine every j <= i.  The predicate alone decides membership, so any span
+ * at least as large as the farthest admitted key gives the same result.
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_attention(int kind, int B, int L, int H, int d_k, int d_v, int P, int dil, int w,
+                     const void *q, const void *k, const void *v, int dt, long nrows,
+                     const long long *rows, long span, double *out) {
+    if (B <= 0 || L <= 0 || H <= 0 || d_k <= 0 || d_v <= 0 || P <= 0 || dil <= 0 || w <= 0)
+        return -1;
+    if (kind != 0 && kind != 1) return -1;
+    const double scale = 1.0 / sqrt((double)d_k);
+
+#pragma omp parallel
+    {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)L);
+        double *qi = (double *)malloc(sizeof(double) * (size_t)d_k);
+#pragma omp for schedule(dynamic, 16)
+        for (long r = 0; r < nrows; ++r) {
+            long long id = rows ? rows[r] : (long long)r;
+            long h = (long)(id % H);
+            long t = (long)((id / H) % L);
+            long b = (long)(id / ((long long)H * L));
+            size_t qoff = (((size_t)b * L + t) * H + h) * d_k;
+            for (int c = 0; c < d_k; ++c) qi[c] = load_elem(q, dt, qoff + c);
+            long lo = (span < 0 || t - span < 0) ? 0 : t - span;
+            double m = -INFINITY;
+            for (long j = lo; j <= t; ++j) {
+                int in = kind == 0 ? swa_in_window(t, j, w) : dswa_in_window(t, j, P, dil, w);
+                if (!in) {
+                    logit[j] = NAN; /* marks a masked key */
+                    continue;
+                }
+                size_t koff = (((size_t)b * L + j) * H + h) * d_k;
+                double s = 0.0;
+                for (int c = 0; c < d_k; ++c) s += qi[c] * load_elem(k, dt, koff + c);
+                s *= scale;
+                logit[j] = s;
+                if (s > m) m = s;
+            }
+            double *o = out + (size_t)r * d_v;
+            for (int c = 0; c < d_v; ++c) o[c] = 0.0;
+            double denom = 0.0;
+            for (long j = lo; j <= t; ++j) {
+                if (isnan(logit[j])) continue;
+                double p = exp(logit[j] - m);
+                denom += p;
+                size_t voff = (((size_t)b * L + j) * H + h) * d_v;
+                for (int c = 0; c < d_v; ++c) o[c] += p * load_elem(v, dt, voff + c);
+            }
+            for (int c = 0; c < d_v; ++c) o[c] /= denom;
+        }
+        free(logit);
+        free(qi);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gated delta memory (section 2.2.1).                                       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * oracle_gdn: the token-by-token recurrence for every (b, h).
+ *
+ * variant 0 (the layer built here): retrieval reads the decayed state,
+ *     v_old = (alpha_t S_{t-1}) k_t                       (Eq. 2 on alpha*S)
+ *     v_new = beta_t v_t + (1 - beta_t) v_old             (Eq. 2)
+ *     S_t   = alpha_t S_{t-1} - v_old k_t^T + v_new k_t^T (Eq. 5)
+ *   which equals alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T.
+ * variant 1 (the equations as printed): v_old = S_{t-1} k_t, then Eq. (2) and
+ *   Eq. (5), i.e. Eq. (6): S_t = alpha_t S_{t-1} + beta_t (v_t - v_old) k_t^T.
+ * matrix_form != 0 evaluates variant 0 as the explicit product
+ *   alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ * (d_k x d_k matrix products), for the self-consistency pin.
+ *
+ * Output (step 4): o_t = S_t q_t, from the updated state.
+ * S0: [B,H,d_v,d_k] or NULL (zero state).  S_out: final state or NULL.
+ * out: [B,L,H,d_v] or NULL.  Returns 0, or -1 on bad arguments.
+ */
+int oracle_gdn(int B, int L, int H, int d_k, int d_v, const void *q, const void *k,
+               const void *v, int dt, const float *alpha, const float *beta,
+               const double *S0, double *S_out, double *out, int variant, int matrix_form) {
+    if (B <= 0 || L < 0 || H <= 0 || d_k <= 0 || d_v <= 0) return -1;
+    if (variant != 0 && variant != 1) return -1;
+    if (matrix_form && variant != 0) return -1;
+
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            size_t sd = (size_t)d_v * d_k;
+            double *S = (double *)malloc(sizeof(double) * sd);
+            double *kt = (double *)malloc(sizeof(double) * d_k);
+            double *qt = (double *)malloc(sizeof(double) * d_k);
+            double *vt = (double *)malloc(sizeof(double) * d_v);
+            double *vold = (double *)malloc(sizeof(double) * d_v);
+            double *G = matrix_form ? (double *)malloc(sizeof(double) * (size_t)d_k * d_k) : NULL;
+            double *T = matrix_form ? (double *)malloc(sizeof(double) * sd) : NULL;
+            if (S0)
+                memcpy(S, S0 + ((size_t)b * H + h) * sd, sizeof(double) * sd);
+            else
+                memset(S, 0, sizeof(double) * sd);
+
+            for (int t = 0; t < L; ++t) {
+                size_t row = ((size_t)b * L + t) * H + h;
+                double a = (double)alpha[row], be = (double)beta[row];
+                for (int c = 0; c < d_k; ++c) {
+                    kt[c] = load_elem(k, dt, row * d_k + c);
+                    qt[c] = load_elem(q, dt, row * d_k + c);
+                }
+                for (int c = 0; c < d_v; ++c) vt[c] = load_elem(v, dt, row * d_v + c);
+
+                if (matrix_form) {
+                    /* G = I - beta k k^T ; T = S G ; S = alpha T + beta v k^T */
+                    for (int i = 0; i < d_k; ++i)
+                        for (int j = 0; j < d_k; ++j)
+                            G[(size_t)i * d_k + j] = (i == j ? 1.0 : 0.0) - be * kt[i] * kt[j];
+                    for (int i = 0; i < d_v; ++i)
+                        for (int j = 0; j < d_k; ++j) {
+                            double s = 0.0;
+                            for (int c = 0; c < d_k; ++c) s += S[(size_t)i * d_k + c] * G[(size_t)c * d_k + j];
+                            T[(size_t)i * d_k + j] = s;
+                        }
+                    for (int i = 0; i < d_v; ++i)
+                        for (int j = 0; j < d_k; ++j)
+                            S[(size_t)i * d_k + j] = a * T[(size_t)i * d_k + j] + be * vt[i] * kt[j];
+                } else {
+                    /* retrieval: v_old = S' k with S' = alpha S (variant 0) or S (variant 1) */
+                    double ret_scale = variant == 0 ? a : 1.0;
+                    for (int i = 0; i < d_v; ++i) {
+                        double s = 0.0;
+                        for (int c = 0; c < d_k; ++c) s += S[(size_t)i * d_k + c] * kt[c];
+                        vold[i] = ret_scale * s;
+                    }
+                    for (int i = 0; i < d_v; ++i) {
+                        double vnew = be * vt[i] + (1.0 - be) * vold[i];
+                        for (int c = 0; c < d_k; ++c) {
+                            double *sij = &S[(size_t)i * d_k + c];
+                            /* decay, remove the old association, write the new one */
+                            *sij = a * (*sij) - vold[i] * kt[c] + vnew * kt[c];
+                        }
+                    }
+                }
+                if (out) {
+                    double *o = out + row * d_v;
+                    for (int i = 0; i < d_v; ++i) {
+                        double s = 0.0;
+                        for (int c = 0; c < d_k; ++c) s += S[(size_t)i * d_k + c] * qt[c];
+                        o[i] = s;
+                    }
+                }
+            }
+            if (S_out) memcpy(S_out + ((size_t)b * H + h) * sd, S, sizeof(double) * sd);
+            free(S);
+            free(kt);
+            free(qt);
+            free(vt);
+            free(vold);
+            free(G);
+            free(T);
+        }
+    }
+    return 0;
+}
+
+/*
+ * oracle_gdn_chunked: variant 0 of oracle_gdn regrouped into chunks of C
+ * tokens.  Not on the pages; derived from the recurrence as follows.  Write
+ * S_t = alpha_t S_{t-1} + u_t k_t^T with u_t = beta_t (v_t - alpha_t S_{t-1} k_t).
+ * Inside a chunk with start state S0 and decay ratios g(t,s) = prod_{s<r<=t}
+ * alpha_r (g(t,s) = exp(l_t - l_s), l = running sum of log alpha, l_0 = 0 at the
+ * chunk start, positions numbered from 1):
+ *   S_t = g(t,0) S0 + sum_{s<=t} g(t,s) u_s k_s^T
+ *   u_t + beta_t sum_{s<t} g(t,s) (k_t . k_s) u_s = beta_t v_t - beta_t g(t,0) S0 k_t
+ *   o_t = g(t,0) S0 q_t + sum_{s<=t} g(t,s) (q_t . k_s) u_s
+ *   S_C = g(C,0) S0 + sum_s g(C,s) u_s k_s^T.
+ * The unit-lower-triangular system for u is solved by forward substitution.
+ * Same arguments as oracle_gdn (variant 0 only).
+ */
+int oracle_gdn_chunked(int B, int L, int H, int d_k, int d_v, const void *q, const void *k,
+                       const void *v, int dt, const float *alpha, const float *beta,
+                       const double *S0, double *S_out, double *out, int C) {
+    if (B <= 0 || L < 0 || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0) return -1;
+
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            size_t sd = (size_t)d_v * d_k;
+            double *S = (double *)malloc(sizeof(double) * sd);
+            double *Kc = (double *)malloc(sizeof(double) * (size_t)C * d_k);
+            double *Qc = (double *)malloc(sizeof(double) * (size_t)C * d_k);
+            double *Vc = (double *)malloc(sizeof(double) * (size_t)C * d_v);
+            double *U = (double *)malloc(sizeof(double) * (size_t)C * d_v);
+            double *ell = (double *)malloc(sizeof(double) * (size_t)(C + 1));
+            double *bt = (double *)malloc(sizeof(double) * (size_t)C);
+            double *Snew = (double *)malloc(sizeof(double) * sd);
+            if (S0)
+                memcpy(S, S0 + ((size_t)b * H + h) * sd, sizeof(double) * sd);
+            else
+                memset(S, 0, sizeof(double) * sd);
+
+            for (int t0 = 0; t0 < L; t0 += C) {
+                int n = (L - t0 < C) ? L - t0 : C;
+                ell[0] = 0.0;
+                for (int i = 0; i < n; ++i) {
+                    size_t row = ((size_t)b * L + t0 + i) * H + h;
+                    ell[i + 1] = ell[i] + log((double)alpha[row]);
+                    bt[i] = (double)beta[row];
+                    for (int c = 0; c < d_k; ++c) {
+                        Kc[(size_t)i * d_k + c] = load_elem(k, dt, row * d_k + c);
+                        Qc[(size_t)i * d_k + c] = load_elem(q, dt, row * d_k + c);
+                    }
+                    for (int c = 0; c < d_v; ++c) Vc[(size_t)i * d_v + c] = load_elem(v, dt, row * d_v + c);
+                }
+                /* forward substitution for u (rows of U) */
+                for (int i = 0; i < n; ++i) {
+                    double g0 = exp(ell[i + 1]);
+                    for (int c = 0; c < d_v; ++c) {
+                        double sk = 0.0;
+                        for (int e = 0; e < d_k; ++e) sk += S[(size_t)c * d_k + e] * Kc[(size_t)i * d_k + e];
+                        U[(size_t)i * d_v + c] = bt[i] * Vc[(size_t)i * d_v + c] - bt[i] * g0 * sk;
+                    }
+                    for (int s = 0; s < i; ++s) {
+                        double kk = 0.0;
+                        for (int e = 0; e < d_k; ++e) kk += Kc[(size_t)i * d_k + e] * Kc[(size_t)s * d_k + e];
+                        double a_is = bt[i] * exp(ell[i + 1] - ell[s + 1]) * kk;
+                        for (int c = 0; c < d_v; ++c) U[(size_t)i * d_v + c] -= a_is * U[(size_t)s * d_v + c];
+                    }
+                }
+                /* outputs */
+                if (out) {
+                    for (int i = 0; i < n; ++i) {
+                        size_t row = ((size_t)b * L + t0 + i) * H + h;
+                        double g0 = exp(ell[i + 1]);
+                        double *o = out + row * d_v;
+                        for (int c = 0; c < d_v; ++c) {
+                            double sq = 0.0;
+                            for (int e = 0; e < d_k; ++e) sq += S[(size_t)c * d_k + e] * Qc[(size_t)i * d_k + e];
+                            o[c] = g0 * sq;
+                        }
+                        for (int s = 0; s <= i; ++s) {
+                            double qk = 0.0;
+                            for (int e = 0; e < d_k; ++e) qk += Qc[(size_t)i * d_k + e] * Kc[(size_t)s * d_k + e];
+                            double coef = exp(ell[i + 1] - ell[s + 1]) * qk;
+                            for (int c = 0; c < d_v; ++c) o[c] += coef * U[(size_t)s * d_v + c];
+                        }
+                    }
+                }
+                /* state at the chunk end */
+                double gC = exp(ell[n]);
+                for (int c = 0; c < d_v; ++c)
+                    for (int e = 0; e < d_k; ++e) {
+                        double s = gC * S[(size_t)c * d_k + e];
+                        for (int i = 0; i < n; ++i)
+                            s += exp(ell[n] - ell[i + 1]) * U[(size_t)i * d_v + c] * Kc[(size_t)i * d_k + e];
+                        Snew[(size_t)c * d_k + e] = s;
+                    }
+                memcpy(S, Snew, sizeof(double) * sd);
+            }
+            if (S_out) memcpy(S_out + ((size_t)b * H + h) * sd, S, sizeof(double) * sd);
+            free(S);
+            free(Kc);
+            free(Qc);
+            free(Vc);
+            free(U);
+            free(ell);
+            free(bt);
+            free(Snew);
+        }
+    }
+    return 0;
+}
+
+/* Number of threads the OpenMP runtime will use (1 without OpenMP). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

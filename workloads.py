@@ -1,0 +1,184 @@
+"""Seeded synthetic inputs for the Hybrid Linear Temporal Attention forward pass.
+
+This module is shared by the fp64 oracle (``oracle/``), the CUDA path
+(``hybrid_linear_temporal_b200``), the tests and ``bench.py``.  It holds the
+workload shapes and the value distributions only -- none of the layer's
+arithmetic -- so that both sides see bit-identical inputs without sharing any
+code of the method itself.
+
+Shapes follow the Kairos paper (arXiv 2606.16533), section 2.2.2: a latent
+video of F frames with P tokens each is flattened to a causal sequence of
+L = F * P tokens, token t = f * P + s.  The synthetic workloads stand in for
+latent video; no dataset is involved.
+
+Distributions (all fp64 draws from ``numpy.random.default_rng(seed)``, drawn in
+the order q, k, v, beta, alpha, gates, then cast once):
+
+* q, k ~ N(0, 1), then L2-normalised per (token, head)
+* v ~ N(0, 1)
+* beta = sigmoid(N(0, 1))
+* alpha = exp(-softplus(N(0, 1) + shift)), shift = 2 (4 for the long-horizon
+  workload); ``alpha_mode="slow"`` is a stress variant with shift = -4
+  (alpha ~ 0.98) that exercises long memory
+* gates ~ U(0, 1) per head, three per head (SWA, DSWA, GDN)
+
+bf16 tensors are stored as ``uint16`` bit patterns (round-to-nearest-even of
+the fp64 draw); ``as_float32`` gives their exact values.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+# Draw block: tensors are generated in blocks of tokens so that the long
+# workloads never hold fp64 copies of the whole tensor.  numpy's Generator
+# continues its stream across calls, so the block size does not change values.
+_BLOCK_TOKENS = 4096
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    d_k: int
+    d_v: int
+    L: int                 # tokens per sequence (one-shot) or total (streaming)
+    P: int                 # tokens per latent frame
+    swa_window: int
+    dswa_window: int
+    dilation: int
+    chunk: int = 64
+    dtype: str = "bf16"    # "bf16" or "fp32"
+    alpha_shift: float = 2.0
+    stream_steps: int = 0  # >0: L tokens arrive in this many equal appends
+    seed: int = 0
+
+    @property
+    def frames(self) -> int:
+        return -(-self.L // self.P)
+
+    @property
+    def step_tokens(self) -> int:
+        return self.L // self.stream_steps if self.stream_steps else self.L
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads: tiny fp32 check, short bf16 clip, the 480P-shaped
+# rollout (headline), streaming rollout and long horizon.
+WORKLOADS = {
+    "tiny_fp32": Workload("tiny_fp32", B=1, H=2, d_k=64, d_v=64, L=256, P=1,
+                          swa_window=32, dswa_window=32, dilation=4, dtype="fp32"),
+    "clip_4k": Workload("clip_4k", B=1, H=16, d_k=128, d_v=128, L=4096, P=256,
+                        swa_window=256, dswa_window=256, dilation=4),
+    "rollout_480p": Workload("rollout_480p", B=1, H=24, d_k=128, d_v=128, L=32760, P=1560,
+                             swa_window=1560, dswa_window=1560, dilation=8),
+    "stream_480p": Workload("stream_480p", B=4, H=24, d_k=128, d_v=128, L=120 * 1560, P=1560,
+                            swa_window=1560, dswa_window=1560, dilation=8, stream_steps=120),
+    "long_131k": Workload("long_131k", B=1, H=24, d_k=128, d_v=128, L=131040, P=1560,
+                          swa_window=1560, dswa_window=3120, dilation=16, alpha_shift=4.0),
+}
+ORDER = ["tiny_fp32", "clip_4k", "rollout_480p", "stream_480p", "long_131k"]
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64/fp32 values to bf16 (nearest, ties to even); return uint16 bits."""
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    rounding = 0x7FFF + ((u >> 16) & 1)
+    return ((u + rounding) >> 16).astype(np.uint16)
+
+
+def bf16_to_float32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+@dataclasses.dataclass
+class Inputs:
+    """Host tensors of one workload.
+
+    q, k: [B, L, H, d_k]; v: [B, L, H, d_v] -- uint16 bf16 bits or float32.
+    alpha, beta: [B, L, H] float32.  gates: [H, 3] float32 (SWA, DSWA, GDN).
+    """
+    wl: Workload
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    alpha: np.ndarray
+    beta: np.ndarray
+    gates: np.ndarray
+
+    def as_float32(self, name: str) -> np.ndarray:
+        a = getattr(self, name)
+        return bf16_to_float32(a) if a.dtype == np.uint16 else a
+
+
+def _normal_tensor(rng, B, L, H, d, normalise, dtype):
+    out = np.empty((B, L, H, d), dtype=np.uint16 if dtype == "bf16" else np.float32)
+    for b in range(B):
+        for t0 in range(0, L, _BLOCK_TOKENS):
+            n = min(_BLOCK_TOKENS, L - t0)
+            x = rng.standard_normal((n, H, d))
+            if normalise:
+                x /= np.linalg.norm(x, axis=-1, keepdims=True)
+            out[b, t0:t0 + n] = bf16_bits(x) if dtype == "bf16" else x.astype(np.float32)
+    return out
+
+
+def make_inputs(wl: Workload, seed: int | None = None, alpha_mode: str = "default",
+                normalise_qk: bool = True) -> Inputs:
+    """Draw the inputs of ``wl`` (see the module docstring for the recipe)."""
+    rng = np.random.default_rng(wl.seed if seed is None else seed)
+    B, L, H = wl.B, wl.L, wl.H
+    q = _normal_tensor(rng, B, L, H, wl.d_k, normalise_qk, wl.dtype)
+    k = _normal_tensor(rng, B, L, H, wl.d_k, normalise_qk, wl.dtype)
+    v = _normal_tensor(rng, B, L, H, wl.d_v, False, wl.dtype)
+    beta = (1.0 / (1.0 + np.exp(-rng.standard_normal((B, L, H))))).astype(np.float32)
+    shift = {"default": wl.alpha_shift, "slow": -4.0}[alpha_mode]
+    z = rng.standard_normal((B, L, H)) + shift
+    softplus = np.logaddexp(0.0, z)
+    alpha = np.exp(-softplus).astype(np.float32)
+    gates = rng.uniform(0.0, 1.0, (H, 3)).astype(np.float32)
+    return Inputs(wl, q, k, v, alpha, beta, gates)
+
+
+def band_pairs(n: int, w: int) -> int:
+    """Number of (query, key) pairs of a causal window of w keys over n tokens."""
+    if n <= w:
+        return n * (n + 1) // 2
+    return w * (w + 1) // 2 + (n - w) * w
+
+
+def dswa_pairs(L: int, P: int, w: int, dilation: int) -> int:
+    """(query, key) pairs of the dilated window: a causal window of w keys over
+    each residue class of frames (frames f = g, g + dilation, ...)."""
+    F = -(-L // P)
+    tot = 0
+    for g in range(dilation):
+        n = sum(min(P, L - f * P) for f in range(g, F, dilation))
+        tot += band_pairs(n, w)
+    return tot
+
+
+def algorithmic_work(wl: Workload) -> dict:
+    """Flops and HBM bytes the method needs for one forward pass of ``wl``.
+
+    Attention: 4 * d flops per in-band (query, key) pair.  GDN: the chunk form,
+    10*C^2*d + 6*C*d^2 + (2/3)*C^3 per chunk of C tokens (d = d_k = d_v).
+    Bytes: q, k, v and out once, alpha and beta once.
+    """
+    eb = 2 if wl.dtype == "bf16" else 4
+    d = wl.d_k
+    B, H, L, C = wl.B, wl.H, wl.L, wl.chunk
+    swa = 4 * d * band_pairs(L, wl.swa_window) * B * H
+    dswa = 4 * d * dswa_pairs(L, wl.P, wl.dswa_window, wl.dilation) * B * H
+    nch = math.ceil(L / C)
+    gdn = nch * (10 * C * C * d + 6 * C * d * d + (2 * C ** 3) // 3) * B * H
+    bytes_ = B * L * H * (3 * d * eb + wl.d_v * eb + 8)
+    return {"swa_flops": swa, "dswa_flops": dswa, "gdn_flops": gdn,
+            "flops": swa + dswa + gdn, "bytes": bytes_,
+            "gdn_bytes": B * L * H * (3 * d * eb + wl.d_v * eb + 8)}
