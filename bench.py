@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the Hybrid Linear Temporal Attention forward pass on B200.
+
+One step = one full layer pass (SWA + DSWA + gated delta memory + gated sum)
+over one batch of the 480P-shaped rollout workload (B=1, H=24, d=128,
+L=32760 = 21 frames x 1560 tokens, windows 1560, dilation 8, bf16), inputs
+resident in HBM.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched by torchrun): every rank runs its own independent sequence
+(weak scaling, no data-path collective); the step time is the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (rank
+0 only), each step a bounded sample of the same workload extrapolated to it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from workloads import WORKLOADS, make_inputs, algorithmic_work  # noqa: E402
+
+METRIC = "hybrid temporal attention fwd tokens/s at L=32760 bf16; % of roofline"
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="rollout_480p")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# process group
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ---------------------------------------------------------------------------
+# roofline
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+KERNEL_SOURCES = {
+    "swa": ["tc_attention.cu"], "dswa": ["tc_attention.cu"], "gdn": ["tc_gdn.cu", "gdn_recurrent.cu"],
+}
+
+
+def source_sha(branch: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[branch]:
+        p = os.path.join(ROOT, "hybrid_linear_temporal_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(branch: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    has not changed since the counters were taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{branch}:{workload}")
+    if not d or d.get("source_sha") != source_sha(branch):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def roofline(branch, ms_per_launch, wl, peaks, sustained=True):
+    work = algorithmic_work(wl)
+    if branch in ("swa", "dswa"):
+        flops = work[f"{branch}_flops"]
+        peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+        ach = flops / (ms_per_launch * 1e-3) / 1e12
+        return {"kernel": f"{branch}_fwd", "bound": "tensor", "achieved": round(ach, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                "traffic": traffic_for(branch, wl.name),
+                "algorithmic": {"flops_per_launch": flops},
+                "peak_kind": f"bf16 dense, {'sustained' if sustained else 'burst'}, {peaks['source']}"}
+    # memory branch: HBM-bound (its q, k, v, alpha, beta read and out write dominate)
+    byts = work["gdn_bytes"]
+    ach = byts / (ms_per_launch * 1e-3) / 1e9
+    return {"kernel": "gdn_fwd", "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+            "traffic": traffic_for("gdn", wl.name),
+            "algorithmic": {"bytes_per_launch": byts, "flops_per_launch": work["gdn_flops"]},
+            "peak_kind": f"HBM copy, {peaks['source']}"}
+
+
+def layer_roofline(ms_step, wl, peaks, sustained=True):
+    work = algorithmic_work(wl)
+    peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * 1e12
+    t_roof = max(work["flops"] / peak, work["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    return {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof / (ms_step * 1e-3), 4),
+            "bound": "tensor" if work["flops"] / peak > work["bytes"] / (peaks["hbm_gbs"] * 1e9) else "hbm",
+            "flops": work["flops"], "bytes": work["bytes"],
+            "peak_kind": f"{'sustained' if sustained else 'burst'} bf16, {peaks['source']}"}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample, extrapolated
+# ---------------------------------------------------------------------------
+def oracle_sample_time(inp, budget_s: float, seed: int = 0):
+    """Seconds the oracle needs for the whole layer on ``inp``'s workload,
+    extrapolated from (a) the memory recurrence of `cores` (batch, head) pairs
+    over a prefix of the sequence and (b) SWA and DSWA rows of random queries.
+    Returns (seconds, cores, sample description)."""
+    import oracle
+    wl = inp.wl
+    cores = oracle.num_threads()
+    nheads = min(cores, wl.H)
+    # (a) memory branch: nheads heads over a prefix
+    t_tok = max(64, min(wl.L, int(2048 * budget_s / 10)))
+    sl = lambda a: np.ascontiguousarray(a[:1, :t_tok, :nheads])
+    t0 = time.perf_counter()
+    oracle.gdn(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.alpha), sl(inp.beta))
+    t_g = time.perf_counter() - t0
+    # scale the prefix so (a) takes about half the budget
+    if t_g < budget_s / 4 and t_tok < wl.L:
+        t_tok = min(wl.L, int(t_tok * (budget_s / 2) / max(t_g, 1e-3)))
+        sl = lambda a: np.ascontiguousarray(a[:1, :t_tok, :nheads])
+        t0 = time.perf_counter()
+        oracle.gdn(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.alpha), sl(inp.beta))
+        t_g = time.perf_counter() - t0
+    per_tokhead_gdn = t_g / (t_tok * nheads) * min(nheads, cores)   # wall time per (token, head) on one core
+    gdn_full = per_tokhead_gdn * wl.B * wl.L * wl.H / min(cores, wl.B * wl.H)
+    # (b) attention rows
+    rng = np.random.default_rng(seed)
+    n = 64
+    times = {}
+    while True:
+        rows = rng.integers(0, wl.B * wl.L * wl.H, size=n)
+        t0 = time.perf_counter()
+        oracle.attention_rows("swa", inp.q, inp.k, inp.v, wl.P, 1, wl.swa_window, rows)
+        t1 = time.perf_counter()
+        oracle.attention_rows("dswa", inp.q, inp.k, inp.v, wl.P, wl.dilation, wl.dswa_window, rows)
+        t2 = time.perf_counter()
+        times = {"swa": (t1 - t0) / n, "dswa": (t2 - t1) / n}
+        if t2 - t0 > budget_s / 4 or n >= 1 << 16:
+            break
+        n = int(n * min(16, max(2, (budget_s / 2) / max(t2 - t0, 1e-3))))
+    attn_full = (times["swa"] + times["dswa"]) * wl.B * wl.L * wl.H
+    desc = (f"memory recurrence: {nheads} heads x {t_tok} tokens; attention: {n} random query rows "
+            f"(SWA and DSWA); extrapolated to B*L*H = {wl.B * wl.L * wl.H} rows")
+    return gdn_full + attn_full, cores, desc
+
+
+def cpu_baseline(inp, budget_s):
+    secs, cores, desc = oracle_sample_time(inp, budget_s)
+    wl = inp.wl
+    return {"value": round(wl.B * wl.L / secs, 3), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle", "sample": desc}
+
+
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    """The oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl)
+    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample_time(inp, per_step, seed=1)
+    total, cores, desc = 0.0, 1, ""
+    for s in range(args.steps):
+        secs, cores, desc = oracle_sample_time(inp, per_step, seed=100 + s)
+        total += secs
+    ms = total / args.steps * 1e3
+    value = wl.B * wl.L / (ms * 1e-3)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, args.gpus),
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, n):
+    return {"workload": wl.name, "B": wl.B, "L": wl.L, "H": wl.H, "d_k": wl.d_k, "d_v": wl.d_v,
+            "tokens_per_frame": wl.P, "swa_window": wl.swa_window, "dswa_window": wl.dswa_window,
+            "dilation": wl.dilation, "chunk": wl.chunk, "global_batch": wl.B * n,
+            "parallelism": f"independent sequences x{n}" if n > 1 else "single GPU",
+            "l2": "inputs larger than L2 (q,k,v,out %.0f MB per step > 126 MB)" % (
+                algorithmic_work(wl)["bytes"] / 1e6)}
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from hybrid_linear_temporal_b200 import HLTA, build
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device")
+    torch.cuda.set_device(local)
+    if not os.path.exists(os.path.join(ROOT, "hybrid_linear_temporal_b200", "libhlta.so")):
+        if rank == 0:
+            build.build()
+        barrier(world)
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl, seed=rank)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+    def dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(a).cuda()
+    d = {n: dev(getattr(inp, n)) for n in ("q", "k", "v", "alpha", "beta", "gates")}
+    out = torch.empty((wl.B, wl.L, wl.H, wl.d_v), dtype=dt, device="cuda")
+    layer = HLTA.for_workload(wl)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["gates"], out=out, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    layer.profile_enable(True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = e0.elapsed_time(e1) / args.steps
+    prof = layer.profile_read()
+    layer.profile_enable(False)
+    ms_max = max_over_ranks(ms, world)
+    value = world * wl.B * wl.L / (ms_max * 1e-3)
+    peaks = measured_peaks()
+
+    branches = {}
+    for b in ("swa", "dswa", "gdn"):
+        p = prof.get(b, {})
+        if p.get("passes"):
+            mpl = p["total_ms"] / p["passes"]
+            branches[b] = {"ms": round(mpl, 4), "roofline": roofline(b, mpl, wl, peaks)}
+    dom = max(branches, key=lambda b: branches[b]["ms"]) if branches else None
+
+    # end to end through the public API with host buffers (pinned)
+    e2e = None
+    if not args.no_e2e:
+        def pin(a):
+            t = torch.from_numpy(a).pin_memory()
+            return t.numpy()
+        hq, hk, hv, ha, hb, hg = (pin(getattr(inp, n)) for n in ("q", "k", "v", "alpha", "beta", "gates"))
+        hout = pin(np.empty((wl.B, wl.L, wl.H, wl.d_v), dtype=inp.v.dtype))
+        layer.forward_host(hq, hk, hv, ha, hb, hg, out=hout)
+        n_e2e = max(3, min(args.steps, 20))
+        barrier(world)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(n_e2e):
+            layer.forward_host(hq, hk, hv, ha, hb, hg, out=hout)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(f0.elapsed_time(f1) / n_e2e, world)
+        h2d = sum(a.nbytes for a in (hq, hk, hv, ha, hb, hg))
+        e2e = {"value": round(world * wl.B * wl.L / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.nbytes),
+               "ms_per_step": round(ms_e2e, 3), "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, args.cpu_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_max, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded, shapes of a 480P latent clip)",
+                "config": config_of(wl, world),
+                "roofline": branches[dom]["roofline"] if dom else None,
+                "layer_roofline": layer_roofline(ms_max, wl, peaks),
+                "branches": branches,
+                "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": int(prof.get("kernel_launches", 0)),
+                "clocks": clk}
+        print(json.dumps(line), flush=True)
+    layer.close()
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,621 @@
+// hlta_api.cu -- the C ABI declared in include/hlta.h: argument checks,
+// handle-owned device memory, and the launch sequence of one layer pass.
+//
+// One pass (Kairos paper, section 2.2) runs the selected branches in the order
+// SWA, DSWA, GDN on the caller's stream.  Each branch kernel adds its gated
+// output g[h,b]*o_b into an fp32 accumulator; the last one selected writes the
+// layer output in the configured dtype (fused gate/sum epilogue).
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <string>
+#include <vector>
+
+#include "hlta.h"
+#include "kernels.h"
+#include "tc_attention.h"
+#include "tc_gdn.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+hlta_status fail(hlta_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+hlta_status ok() {
+    g_last_error.clear();
+    return HLTA_OK;
+}
+
+// Host-side failure injection for tests: HLTA_INJECT_FAIL=<entry point name>
+// (or "all") makes that entry point fail with HLTA_ERR_INJECTED before doing
+// anything.
+bool injected(const char *fn) {
+    const char *e = getenv("HLTA_INJECT_FAIL");
+    if (!e || !*e) return false;
+    return strcmp(e, "all") == 0 || strcmp(e, fn) == 0;
+}
+
+#define INJECT(fn)                                                        \
+    do {                                                                  \
+        if (injected(fn)) return fail(HLTA_ERR_INJECTED, "%s: injected failure", fn); \
+    } while (0)
+
+#define CK(call)                                                                          \
+    do {                                                                                  \
+        cudaError_t e_ = (call);                                                          \
+        if (e_ != cudaSuccess)                                                            \
+            return fail(HLTA_ERR_CUDA, "%s:%d %s: %s", __FILE__, __LINE__, #call,        \
+                        cudaGetErrorString(e_));                                          \
+    } while (0)
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct hlta_handle {
+    hlta_config cfg;
+    int device = 0;
+    int elem_bytes = 2;
+    long long acc_rows = 0;      // token rows per batch the accumulator holds
+    float *acc = nullptr;        // [B, acc_rows, H, d_v]
+    int *dev_err = nullptr;      // device error word
+    // streaming state
+    float *S_stream = nullptr;   // [B, H, d_v, d_k]
+    void *ring_k = nullptr;      // [B, ring_cap, H, d_k]
+    void *ring_v = nullptr;      // [B, ring_cap, H, d_v]
+    long long ring_cap = 0;
+    long long pos = 0;
+    long long hdr[8] = {0};
+    // staging for hlta_forward_host
+    char *stage = nullptr;
+    size_t stage_bytes = 0;
+    hlta::TcAttention *tc_attn = nullptr;
+    hlta::TcGdn *tc_gdn = nullptr;
+    // profiling (hlta_profile_enable)
+    bool prof = false;
+    struct Mark {
+        int slot;
+        cudaEvent_t a, b;
+    };
+    std::vector<Mark> marks;
+    std::vector<cudaEvent_t> event_pool;
+    double prof_ms[3] = {0, 0, 0};
+    long long prof_passes[3] = {0, 0, 0};
+    long long prof_launches = 0;
+};
+
+namespace {
+
+constexpr long long kCkptMagic = 0x484c544143503031LL;  // "HLTACP01"
+constexpr size_t kCkptHeader = 256;
+
+size_t state_elems(const hlta_config &c) { return (size_t)c.B * c.H * c.d_v * c.d_k; }
+
+// Farthest key (in tokens, behind the query) any window can admit.
+long long max_lookback(const hlta_config &c) {
+    const long long P = c.tokens_per_frame;
+    const long long swa = c.swa_window - 1;
+    // DSWA: i - j = dil*g*P + s_i - s_j with r(i) - r(j) = g*P + s_i - s_j < w and
+    // g*P <= w - 1 + P - 1, so i - j <= (dil - 1)*g_max*P + w - 1.
+    const long long gmax = (c.dswa_window + P - 2) / P;
+    const long long dswa = (long long)(c.dswa_dilation - 1) * gmax * P + c.dswa_window - 1;
+    return swa > dswa ? swa : dswa;
+}
+
+hlta_status check_config(const hlta_config *c) {
+    if (!c) return fail(HLTA_ERR_INVALID_ARG, "hlta_create: cfg is NULL");
+    if (c->B < 1 || c->H < 1) return fail(HLTA_ERR_INVALID_ARG, "B and H must be >= 1");
+    if (c->d_k < 1 || c->d_v < 1) return fail(HLTA_ERR_INVALID_ARG, "d_k and d_v must be >= 1");
+    if (c->tokens_per_frame < 1) return fail(HLTA_ERR_INVALID_ARG, "tokens_per_frame must be >= 1");
+    if (c->swa_window < 1 || c->dswa_window < 1)
+        return fail(HLTA_ERR_INVALID_ARG, "windows must be >= 1");
+    if (c->dswa_dilation < 1) return fail(HLTA_ERR_INVALID_ARG, "dswa_dilation must be >= 1");
+    if (c->dtype != HLTA_BF16 && c->dtype != HLTA_FP32)
+        return fail(HLTA_ERR_INVALID_ARG, "dtype must be HLTA_BF16 or HLTA_FP32");
+    if (c->max_seq_len < 1) return fail(HLTA_ERR_INVALID_ARG, "max_seq_len must be >= 1");
+    if (c->max_stream_tokens < 0) return fail(HLTA_ERR_INVALID_ARG, "max_stream_tokens must be >= 0");
+    if ((c->d_k != 64 && c->d_k != 128) || (c->d_v != 64 && c->d_v != 128))
+        return fail(HLTA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128");
+    if (c->chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64");
+    const long long big = 1LL << 31;
+    if ((long long)c->B * c->max_seq_len * c->H >= big / 128)
+        return fail(HLTA_ERR_UNSUPPORTED, "B*max_seq_len*H too large");
+    return HLTA_OK;
+}
+
+struct Inputs {
+    const void *q, *k, *v;
+    const float *alpha, *beta, *gates;
+};
+
+hlta_status check_inputs(const char *fn, const Inputs &in, const void *out) {
+    const void *ptrs[] = {in.q, in.k, in.v, in.alpha, in.beta, in.gates, out};
+    const char *names[] = {"q", "k", "v", "alpha", "beta", "gates", "out"};
+    for (int i = 0; i < 7; ++i) {
+        if (!ptrs[i]) return fail(HLTA_ERR_INVALID_ARG, "%s: %s is NULL", fn, names[i]);
+        if (!aligned16(ptrs[i]))
+            return fail(HLTA_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, names[i]);
+    }
+    return HLTA_OK;
+}
+
+cudaEvent_t pooled_event(hlta_handle *h) {
+    if (!h->event_pool.empty()) {
+        cudaEvent_t e = h->event_pool.back();
+        h->event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Brackets one branch's launches with events when profiling is on.
+struct ProfScope {
+    hlta_handle *h;
+    int slot;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    ProfScope(hlta_handle *h_, int slot_, cudaStream_t s_) : h(h_), slot(slot_), s(s_) {
+        if (!h->prof) return;
+        a = pooled_event(h);
+        b = pooled_event(h);
+        if (a && b) cudaEventRecord(a, s);
+    }
+    void done(int launches) {
+        if (!h->prof || !a || !b) return;
+        cudaEventRecord(b, s);
+        h->marks.push_back({slot, a, b});
+        h->prof_launches += launches;
+    }
+};
+
+// Output mode of the idx-th of n selected branches.
+int out_mode(int idx, int n) {
+    if (n == 1) return hlta::OUT_FINAL_ONLY;
+    if (idx == 0) return hlta::OUT_STORE;
+    return idx == n - 1 ? hlta::OUT_FINAL : hlta::OUT_ADD;
+}
+
+// Run the selected branches of one pass.
+//   nq queries at absolute positions pos0 .. pos0+nq-1 (q, alpha, beta, k, v of
+//   those tokens: [B, nq, ...]); keys/values are read from (kst, vst) with
+//   key_rows rows per batch (position p at row p % key_rows).
+hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, const void *kst,
+                     const void *vst, long long key_rows, bool one_shot, const float *S_in,
+                     float *S_out, void *out, unsigned branches, cudaStream_t s) {
+    const hlta_config &c = h->cfg;
+    const bool bf16 = c.dtype == HLTA_BF16;
+    int sel[3], n = 0;
+    for (int b = 0; b < 3; ++b)
+        if (branches & (1u << b)) sel[n++] = b;
+    if (n == 0) {
+        CK(cudaMemsetAsync(out, 0, (size_t)c.B * nq * c.H * c.d_v * h->elem_bytes, s));
+        return HLTA_OK;
+    }
+    for (int idx = 0; idx < n; ++idx) {
+        const int br = sel[idx];
+        const int mode = out_mode(idx, n);
+        ProfScope ps(h, br, s);
+        int launches = 1;
+        if (br == 0 || br == 1) {
+            hlta::WindowGeom g;
+            g.P = c.tokens_per_frame;
+            g.dil = br == 0 ? 1 : c.dswa_dilation;
+            g.w = br == 0 ? c.swa_window : c.dswa_window;
+            bool done = false;
+            if (one_shot && h->tc_attn) {
+                cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, g, in.gates, br, mode, h->acc,
+                                                out, h->dev_err, s, &done);
+                if (e != cudaSuccess)
+                    return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
+            }
+            if (!done) {
+                hlta::AttnSimtArgs a;
+                a.q = in.q;
+                a.k = kst;
+                a.v = vst;
+                a.q_pos0 = pos0;
+                a.nq = nq;
+                a.B = c.B;
+                a.H = c.H;
+                a.d_k = c.d_k;
+                a.d_v = c.d_v;
+                a.key_rows = key_rows;
+                a.geom = g;
+                a.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d_k);
+                a.gates = in.gates;
+                a.gate_col = br;
+                a.out_mode = mode;
+                a.acc = h->acc;
+                a.out = out;
+                CK(hlta::launch_attn_simt(a, bf16, s));
+            }
+        } else {
+            bool done = false;
+            if (h->tc_gdn) {
+                cudaError_t e = h->tc_gdn->run(in.q, in.k, in.v, in.alpha, in.beta, nq, S_in, S_out,
+                                               in.gates, mode, h->acc, out, h->dev_err, s, &done,
+                                               &launches);
+                if (e != cudaSuccess)
+                    return fail(HLTA_ERR_CUDA, "tensor-core memory: %s", cudaGetErrorString(e));
+            }
+            if (!done) {
+                hlta::GdnRecArgs a;
+                a.q = in.q;
+                a.k = in.k;
+                a.v = in.v;
+                a.alpha = in.alpha;
+                a.beta = in.beta;
+                a.S_in = S_in;
+                a.S_out = S_out;
+                a.n = nq;
+                a.B = c.B;
+                a.H = c.H;
+                a.d_k = c.d_k;
+                a.d_v = c.d_v;
+                a.gates = in.gates;
+                a.out_mode = mode;
+                a.acc = h->acc;
+                a.out = out;
+                CK(hlta::launch_gdn_recurrent(a, bf16, s));
+            }
+        }
+        ps.done(launches);
+    }
+    return HLTA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hlta_version(void) { return 100; }
+
+const char *hlta_last_error(void) { return g_last_error.c_str(); }
+
+hlta_status hlta_create(const hlta_config *cfg, hlta_handle **out) {
+    INJECT("hlta_create");
+    if (!out) return fail(HLTA_ERR_INVALID_ARG, "hlta_create: out is NULL");
+    *out = nullptr;
+    hlta_status st = check_config(cfg);
+    if (st != HLTA_OK) return st;
+
+    int dev = 0;
+    CK(cudaGetDevice(&dev));
+    cudaDeviceProp prop;
+    CK(cudaGetDeviceProperties(&prop, dev));
+    if (prop.major != 10)
+        return fail(HLTA_ERR_CUDA, "hlta_create: device %d is sm_%d%d; this build targets sm_100a",
+                    dev, prop.major, prop.minor);
+
+    hlta_handle *h = new hlta_handle();
+    h->cfg = *cfg;
+    h->device = dev;
+    h->elem_bytes = cfg->dtype == HLTA_BF16 ? 2 : 4;
+    h->acc_rows = cfg->max_seq_len > cfg->max_stream_tokens ? cfg->max_seq_len : cfg->max_stream_tokens;
+
+    auto alloc = [&](void **p, size_t bytes) -> bool {
+        if (cudaMalloc(p, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        return true;
+    };
+    const size_t acc_bytes = (size_t)cfg->B * h->acc_rows * cfg->H * cfg->d_v * sizeof(float);
+    bool okk = alloc((void **)&h->acc, acc_bytes) && alloc((void **)&h->dev_err, sizeof(int));
+    if (okk && cfg->max_stream_tokens > 0) {
+        long long cap = cfg->max_stream_tokens + max_lookback(*cfg);
+        cap = (cap + 127) / 128 * 128;
+        h->ring_cap = cap;
+        okk = alloc((void **)&h->S_stream, state_elems(*cfg) * sizeof(float)) &&
+              alloc(&h->ring_k, (size_t)cfg->B * cap * cfg->H * cfg->d_k * h->elem_bytes) &&
+              alloc(&h->ring_v, (size_t)cfg->B * cap * cfg->H * cfg->d_v * h->elem_bytes);
+    }
+    if (!okk) {
+        hlta_destroy(h);
+        return fail(HLTA_ERR_OOM, "hlta_create: device allocation failed");
+    }
+    if (cudaMemset(h->dev_err, 0, sizeof(int)) != cudaSuccess ||
+        (h->S_stream && cudaMemset(h->S_stream, 0, state_elems(*cfg) * sizeof(float)) != cudaSuccess)) {
+        hlta_destroy(h);
+        return fail(HLTA_ERR_CUDA, "hlta_create: cudaMemset failed");
+    }
+    if (cfg->dtype == HLTA_BF16) {
+        h->tc_attn = hlta::TcAttention::create(*cfg, h->acc_rows);
+        h->tc_gdn = hlta::TcGdn::create(*cfg, cfg->max_seq_len);
+    }
+    *out = h;
+    return ok();
+}
+
+hlta_status hlta_destroy(hlta_handle *h) {
+    if (!h) return ok();
+    cudaSetDevice(h->device);
+    cudaDeviceSynchronize();
+    cudaFree(h->acc);
+    cudaFree(h->dev_err);
+    cudaFree(h->S_stream);
+    cudaFree(h->ring_k);
+    cudaFree(h->ring_v);
+    cudaFree(h->stage);
+    for (auto &m : h->marks) {
+        cudaEventDestroy(m.a);
+        cudaEventDestroy(m.b);
+    }
+    for (auto e : h->event_pool) cudaEventDestroy(e);
+    delete h->tc_attn;
+    delete h->tc_gdn;
+    delete h;
+    return ok();
+}
+
+hlta_status hlta_forward(hlta_handle *h, int L, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta, const float *gates, const float *S0,
+                         float *S_out, void *out, unsigned branches, void *stream) {
+    INJECT("hlta_forward");
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_forward: handle is NULL");
+    if (L < 1 || L > h->cfg.max_seq_len)
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_forward: L=%d outside [1, max_seq_len=%d]", L,
+                    h->cfg.max_seq_len);
+    if (branches & ~7u) return fail(HLTA_ERR_INVALID_ARG, "hlta_forward: unknown branch bits");
+    if (branches == 0) branches = HLTA_BRANCH_ALL;
+    Inputs in{q, k, v, alpha, beta, gates};
+    hlta_status st = check_inputs("hlta_forward", in, out);
+    if (st != HLTA_OK) return st;
+    if ((S0 && !aligned16(S0)) || (S_out && !aligned16(S_out)))
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_forward: S0/S_out not 16-byte aligned");
+    CK(cudaSetDevice(h->device));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = run_pass(h, in, 0, L, k, v, L, true, S0, (branches & HLTA_BRANCH_GDN) ? S_out : nullptr,
+                  out, branches, s);
+    if (st != HLTA_OK) return st;
+    CK(cudaGetLastError());
+    return ok();
+}
+
+hlta_status hlta_forward_host(hlta_handle *h, int L, const void *q, const void *k, const void *v,
+                              const float *alpha, const float *beta, const float *gates,
+                              const float *S0, float *S_out, void *out, unsigned branches,
+                              void *stream) {
+    INJECT("hlta_forward_host");
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_forward_host: handle is NULL");
+    const hlta_config &c = h->cfg;
+    if (L < 1 || L > c.max_seq_len)
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_forward_host: L=%d outside [1, %d]", L, c.max_seq_len);
+    if (!q || !k || !v || !alpha || !beta || !gates || !out)
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_forward_host: a required pointer is NULL");
+    CK(cudaSetDevice(h->device));
+    const size_t eb = h->elem_bytes;
+    auto up16 = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t rows_max = (size_t)c.B * c.max_seq_len * c.H;
+    const size_t nq = up16(rows_max * c.d_k * eb), nv = up16(rows_max * c.d_v * eb);
+    const size_t ng = up16(rows_max * sizeof(float)), nh = up16((size_t)c.H * 3 * sizeof(float));
+    const size_t ns = up16(state_elems(c) * sizeof(float));
+    const size_t need = 2 * nq + 2 * nv + 2 * ng + nh + 2 * ns;
+    if (!h->stage) {
+        if (cudaMalloc((void **)&h->stage, need) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(HLTA_ERR_OOM, "hlta_forward_host: staging allocation failed");
+        }
+        h->stage_bytes = need;
+    }
+    char *p = h->stage;
+    void *dq = p; p += nq;
+    void *dk = p; p += nq;
+    void *dv = p; p += nv;
+    void *dout = p; p += nv;
+    float *da = (float *)p; p += ng;
+    float *db = (float *)p; p += ng;
+    float *dg = (float *)p; p += nh;
+    float *dS0 = (float *)p; p += ns;
+    float *dS1 = (float *)p;
+    const size_t rows = (size_t)c.B * L * c.H;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CK(cudaMemcpyAsync(dq, q, rows * c.d_k * eb, cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(dk, k, rows * c.d_k * eb, cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(dv, v, rows * c.d_v * eb, cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(da, alpha, rows * sizeof(float), cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(db, beta, rows * sizeof(float), cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(dg, gates, (size_t)c.H * 3 * sizeof(float), cudaMemcpyHostToDevice, s));
+    if (S0) CK(cudaMemcpyAsync(dS0, S0, state_elems(c) * sizeof(float), cudaMemcpyHostToDevice, s));
+    hlta_status st = hlta_forward(h, L, dq, dk, dv, da, db, dg, S0 ? dS0 : nullptr,
+                                  S_out ? dS1 : nullptr, dout, branches, stream);
+    if (st != HLTA_OK) return st;
+    CK(cudaMemcpyAsync(out, dout, rows * c.d_v * eb, cudaMemcpyDeviceToHost, s));
+    if (S_out) CK(cudaMemcpyAsync(S_out, dS1, state_elems(c) * sizeof(float), cudaMemcpyDeviceToHost, s));
+    CK(cudaStreamSynchronize(s));
+    return ok();
+}
+
+hlta_status hlta_stream_step(hlta_handle *h, int n, const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta, const float *gates, void *out,
+                             unsigned branches, void *stream) {
+    INJECT("hlta_stream_step");
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_step: handle is NULL");
+    if (h->cfg.max_stream_tokens < 1)
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_step: handle created with max_stream_tokens = 0");
+    if (n < 1 || n > h->cfg.max_stream_tokens)
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_step: n=%d outside [1, %d]", n,
+                    h->cfg.max_stream_tokens);
+    if (branches & ~7u) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_step: unknown branch bits");
+    if (branches == 0) branches = HLTA_BRANCH_ALL;
+    Inputs in{q, k, v, alpha, beta, gates};
+    hlta_status st = check_inputs("hlta_stream_step", in, out);
+    if (st != HLTA_OK) return st;
+    CK(cudaSetDevice(h->device));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const hlta_config &c = h->cfg;
+    hlta::RingAppendArgs ra;
+    ra.k = k;
+    ra.v = v;
+    ra.ring_k = h->ring_k;
+    ra.ring_v = h->ring_v;
+    ra.pos0 = h->pos;
+    ra.cap = h->ring_cap;
+    ra.n = n;
+    ra.B = c.B;
+    ra.H = c.H;
+    ra.d_k = c.d_k;
+    ra.d_v = c.d_v;
+    ra.elem_bytes = h->elem_bytes;
+    CK(hlta::launch_ring_append(ra, s));
+    if (h->prof) h->prof_launches += 2;
+    st = run_pass(h, in, h->pos, n, h->ring_k, h->ring_v, h->ring_cap, false, h->S_stream,
+                  h->S_stream, out, branches, s);
+    if (st != HLTA_OK) return st;
+    CK(cudaGetLastError());
+    h->pos += n;
+    return ok();
+}
+
+hlta_status hlta_state_get(hlta_handle *h, float *S_dst, long long *pos_out, void *stream) {
+    INJECT("hlta_state_get");
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_state_get: handle is NULL");
+    if (!h->S_stream) return fail(HLTA_ERR_INVALID_ARG, "hlta_state_get: streaming disabled");
+    if (!S_dst) return fail(HLTA_ERR_INVALID_ARG, "hlta_state_get: S_dst is NULL");
+    CK(cudaSetDevice(h->device));
+    CK(cudaMemcpyAsync(S_dst, h->S_stream, state_elems(h->cfg) * sizeof(float),
+                       cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+    if (pos_out) *pos_out = h->pos;
+    return ok();
+}
+
+hlta_status hlta_stream_reset(hlta_handle *h, void *stream) {
+    INJECT("hlta_stream_reset");
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_reset: handle is NULL");
+    if (!h->S_stream) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_reset: streaming disabled");
+    CK(cudaSetDevice(h->device));
+    CK(cudaMemsetAsync(h->S_stream, 0, state_elems(h->cfg) * sizeof(float),
+                       static_cast<cudaStream_t>(stream)));
+    h->pos = 0;
+    return ok();
+}
+
+long long hlta_stream_checkpoint_bytes(const hlta_handle *h) {
+    if (!h || !h->S_stream) return 0;
+    const hlta_config &c = h->cfg;
+    return (long long)(kCkptHeader + state_elems(c) * sizeof(float) +
+                       (size_t)c.B * h->ring_cap * c.H * (c.d_k + c.d_v) * h->elem_bytes);
+}
+
+hlta_status hlta_stream_save(hlta_handle *h, void *dst, void *stream) {
+    INJECT("hlta_stream_save");
+    if (!h || !dst) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_save: NULL argument");
+    if (!h->S_stream) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_save: streaming disabled");
+    CK(cudaSetDevice(h->device));
+    const hlta_config &c = h->cfg;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    h->hdr[0] = kCkptMagic;
+    h->hdr[1] = h->pos;
+    h->hdr[2] = h->ring_cap;
+    h->hdr[3] = hlta_stream_checkpoint_bytes(h);
+    h->hdr[4] = ((long long)c.B << 40) ^ ((long long)c.H << 24) ^ (c.d_k << 12) ^ c.d_v;
+    char *d = static_cast<char *>(dst);
+    CK(cudaMemcpyAsync(d, h->hdr, sizeof h->hdr, cudaMemcpyHostToDevice, s));
+    CK(cudaStreamSynchronize(s));  // hdr is pageable host memory reused by later calls
+    d += kCkptHeader;
+    const size_t sb = state_elems(c) * sizeof(float);
+    CK(cudaMemcpyAsync(d, h->S_stream, sb, cudaMemcpyDeviceToDevice, s));
+    d += sb;
+    const size_t kb = (size_t)c.B * h->ring_cap * c.H * c.d_k * h->elem_bytes;
+    const size_t vb = (size_t)c.B * h->ring_cap * c.H * c.d_v * h->elem_bytes;
+    CK(cudaMemcpyAsync(d, h->ring_k, kb, cudaMemcpyDeviceToDevice, s));
+    CK(cudaMemcpyAsync(d + kb, h->ring_v, vb, cudaMemcpyDeviceToDevice, s));
+    return ok();
+}
+
+hlta_status hlta_stream_load(hlta_handle *h, const void *src, void *stream) {
+    INJECT("hlta_stream_load");
+    if (!h || !src) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_load: NULL argument");
+    if (!h->S_stream) return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_load: streaming disabled");
+    CK(cudaSetDevice(h->device));
+    const hlta_config &c = h->cfg;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    long long hdr[8];
+    CK(cudaMemcpyAsync(hdr, src, sizeof hdr, cudaMemcpyDeviceToHost, s));
+    CK(cudaStreamSynchronize(s));
+    const long long sig = ((long long)c.B << 40) ^ ((long long)c.H << 24) ^ (c.d_k << 12) ^ c.d_v;
+    if (hdr[0] != kCkptMagic || hdr[2] != h->ring_cap || hdr[3] != hlta_stream_checkpoint_bytes(h) ||
+        hdr[4] != sig)
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_stream_load: checkpoint does not match this handle");
+    const char *d = static_cast<const char *>(src) + kCkptHeader;
+    const size_t sb = state_elems(c) * sizeof(float);
+    CK(cudaMemcpyAsync(h->S_stream, d, sb, cudaMemcpyDeviceToDevice, s));
+    d += sb;
+    const size_t kb = (size_t)c.B * h->ring_cap * c.H * c.d_k * h->elem_bytes;
+    const size_t vb = (size_t)c.B * h->ring_cap * c.H * c.d_v * h->elem_bytes;
+    CK(cudaMemcpyAsync(h->ring_k, d, kb, cudaMemcpyDeviceToDevice, s));
+    CK(cudaMemcpyAsync(h->ring_v, d + kb, vb, cudaMemcpyDeviceToDevice, s));
+    h->pos = hdr[1];
+    return ok();
+}
+
+hlta_status hlta_profile_enable(hlta_handle *h, int enable) {
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_profile_enable: handle is NULL");
+    CK(cudaSetDevice(h->device));
+    CK(cudaDeviceSynchronize());
+    for (auto &m : h->marks) {
+        h->event_pool.push_back(m.a);
+        h->event_pool.push_back(m.b);
+    }
+    h->marks.clear();
+    for (int i = 0; i < 3; ++i) {
+        h->prof_ms[i] = 0;
+        h->prof_passes[i] = 0;
+    }
+    h->prof_launches = 0;
+    h->prof = enable != 0;
+    return ok();
+}
+
+hlta_status hlta_profile_read(hlta_handle *h, hlta_profile_data *out) {
+    if (!h || !out) return fail(HLTA_ERR_INVALID_ARG, "hlta_profile_read: NULL argument");
+    CK(cudaSetDevice(h->device));
+    CK(cudaDeviceSynchronize());
+    for (auto &m : h->marks) {
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, m.a, m.b));
+        h->prof_ms[m.slot] += ms;
+        h->prof_passes[m.slot] += 1;
+        h->event_pool.push_back(m.a);
+        h->event_pool.push_back(m.b);
+    }
+    h->marks.clear();
+    memset(out, 0, sizeof *out);
+    out->count = 3;
+    const char *names[3] = {"swa", "dswa", "gdn"};
+    for (int i = 0; i < 3; ++i) {
+        snprintf(out->name[i], sizeof out->name[i], "%s", names[i]);
+        out->total_ms[i] = h->prof_ms[i];
+        out->passes[i] = h->prof_passes[i];
+    }
+    out->kernel_launches = h->prof_launches;
+    return ok();
+}
+
+hlta_status hlta_device_status(hlta_handle *h) {
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_device_status: handle is NULL");
+    CK(cudaSetDevice(h->device));
+    CK(cudaDeviceSynchronize());
+    int e = 0;
+    CK(cudaMemcpy(&e, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost));
+    if (e != hlta::DEVERR_NONE) {
+        CK(cudaMemset(h->dev_err, 0, sizeof(int)));
+        return fail(HLTA_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (code %d)", e);
+    }
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,23 @@
+// tc_attention.h -- tensor-core (tcgen05) sliding-window attention for bf16.
+#pragma once
+#include <cuda_runtime.h>
+
+#include "hlta.h"
+#include "kernels.h"
+
+namespace hlta {
+
+class TcAttention {
+public:
+    // Returns nullptr when the configuration has no tensor-core path.
+    static TcAttention *create(const hlta_config &cfg, long long max_rows);
+    virtual ~TcAttention() {}
+    // One branch (gate_col 0 = SWA, 1 = DSWA) over a full sequence of L tokens.
+    // Sets *done = false (and enqueues nothing) when this case is not covered,
+    // so the caller runs the CUDA-core kernel instead.
+    virtual cudaError_t run(const void *q, const void *k, const void *v, int L, WindowGeom g,
+                            const float *gates, int gate_col, int mode, float *acc, void *out,
+                            int *dev_err, cudaStream_t s, bool *done) = 0;
+};
+
+}  // namespace hlta

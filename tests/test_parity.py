@@ -1,0 +1,231 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle on
+the same seeded inputs.
+
+Tolerances: bf16 -- max abs error <= 2e-2 and relative L2 <= 5e-3; fp32 --
+relative L2 <= 1e-4.  Small workloads are compared element by element; the
+full-size workloads on sampled rows (frame boundaries, window edges, first and
+last tokens plus random rows) with the memory branch checked on every row.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import WORKLOADS, make_inputs
+from parity_util import (to_device, to_numpy64, run_gpu, sample_rows, oracle_rows, assert_close,
+                         errors)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from hybrid_linear_temporal_b200 import build
+    build.build()
+    return torch
+
+
+def layer_for(wl, **kw):
+    from hybrid_linear_temporal_b200 import HLTA
+    return HLTA.for_workload(wl, **kw)
+
+
+def full_compare(torch_cuda, wl, seed=0, alpha_mode="default", normalise_qk=True, S0=None):
+    inp = make_inputs(wl, seed=seed, alpha_mode=alpha_mode, normalise_qk=normalise_qk)
+    ref = oracle.forward(inp, S0=S0)
+    layer = layer_for(wl)
+    dev = to_device(inp)
+    S0_dev = None if S0 is None else torch_cuda.from_numpy(S0.astype(np.float32)).cuda()
+    out, S = run_gpu(layer, dev, S0=S0_dev, want_state=True)
+    got = to_numpy64(out)
+    e = assert_close(got, ref["out"], wl.dtype, f"{wl.name} layer")
+    assert_close(to_numpy64(S), ref["S"], "fp32" if wl.dtype == "fp32" else "bf16", f"{wl.name} state")
+    for i, name in enumerate(("swa", "dswa", "gdn")):
+        o, _ = run_gpu(layer, dev, S0=S0_dev, branches=1 << i)
+        g = inp.gates[None, None, :, i, None].astype(np.float64)
+        assert_close(to_numpy64(o), g * ref[name], wl.dtype, f"{wl.name} branch {name}")
+    layer.close()
+    return e
+
+
+def test_tiny_fp32(torch_cuda):
+    full_compare(torch_cuda, WORKLOADS["tiny_fp32"])
+
+
+def test_clip_4k_bf16(torch_cuda):
+    full_compare(torch_cuda, WORKLOADS["clip_4k"])
+
+
+@pytest.mark.parametrize("case", [
+    dict(L=1), dict(L=63), dict(L=65), dict(L=200, P=16), dict(L=333, P=50),
+    dict(L=256, swa_window=1, dswa_window=1), dict(L=300, swa_window=1000, dswa_window=1000),
+    dict(L=256, dilation=1), dict(L=384, P=8, dilation=5, dswa_window=40),
+    dict(L=512, d_k=64, d_v=64), dict(B=2, L=192, H=3), dict(L=640, P=128, swa_window=300),
+])
+def test_edge_cases_bf16(torch_cuda, case):
+    base = WORKLOADS["clip_4k"].with_(H=2, L=256, P=32, swa_window=48, dswa_window=40, dilation=3)
+    full_compare(torch_cuda, base.with_(**case))
+
+
+@pytest.mark.parametrize("case", [dict(L=1), dict(L=100, P=7), dict(L=130, d_k=128, d_v=64)])
+def test_edge_cases_fp32(torch_cuda, case):
+    full_compare(torch_cuda, WORKLOADS["tiny_fp32"].with_(**case))
+
+
+def test_initial_state_and_stress_inputs(torch_cuda):
+    wl = WORKLOADS["clip_4k"].with_(H=4, L=1024, P=64, swa_window=100, dswa_window=80, dilation=4)
+    S0 = np.random.default_rng(3).standard_normal((1, 4, 128, 128)) * 0.1
+    full_compare(torch_cuda, wl, S0=S0)
+    full_compare(torch_cuda, wl, seed=1, alpha_mode="slow")
+    full_compare(torch_cuda, wl, seed=2, normalise_qk=False)
+
+
+def _sampled_compare(torch_cuda, wl, n_rows, heads_for_state=None):
+    inp = make_inputs(wl)
+    layer = layer_for(wl)
+    dev = to_device(inp)
+    out, S = run_gpu(layer, dev, want_state=True)
+    got = to_numpy64(out).reshape(-1, wl.d_v)
+    rows = sample_rows(wl, n_rows)
+    gdn_out, S_ref = oracle.gdn(inp.q, inp.k, inp.v, inp.alpha, inp.beta)
+    ref = oracle_rows(inp, rows, gdn_out=gdn_out)
+    assert_close(got[rows], ref, wl.dtype, f"{wl.name} sampled rows")
+    # the memory branch on every row
+    o, _ = run_gpu(layer, dev, branches=4)
+    g = inp.gates[None, None, :, 2, None].astype(np.float64)
+    assert_close(to_numpy64(o), g * gdn_out, wl.dtype, f"{wl.name} memory branch, all rows")
+    assert_close(to_numpy64(S), S_ref, wl.dtype, f"{wl.name} final state")
+    layer.close()
+    return inp, to_numpy64(S)
+
+
+def test_rollout_480p_bf16(torch_cuda):
+    _sampled_compare(torch_cuda, WORKLOADS["rollout_480p"], 3000)
+
+
+@pytest.mark.slow
+def test_long_131k_bf16(torch_cuda):
+    """Long horizon: sampled rows, the memory on every row, and the state norm
+    stays within the contraction bound sup ||S|| <= max(beta |v|) / (1 - max alpha)."""
+    inp, S = _sampled_compare(torch_cuda, WORKLOADS["long_131k"], 2000)
+    vn = np.linalg.norm(inp.as_float32("v").astype(np.float64), axis=-1)
+    bound = (inp.beta * vn).max() / (1 - inp.alpha.max())
+    assert np.linalg.norm(S, axis=(-2, -1)).max() <= bound
+
+
+def test_stream_equals_one_shot_and_oracle(torch_cuda):
+    """Streaming appends (ring + carried state) vs the oracle's one-shot pass
+    over the concatenation, at a reduced size of the streaming workload."""
+    torch = torch_cuda
+    wl = WORKLOADS["stream_480p"].with_(B=2, H=4, L=12 * 96, P=96, swa_window=96,
+                                        dswa_window=96, dilation=4, stream_steps=12)
+    _stream_check(torch, wl, n_rows=1500)
+
+
+def _stream_check(torch, wl, n_rows, heads=None):
+    from hybrid_linear_temporal_b200 import HLTA
+    inp = make_inputs(wl)
+    n = wl.step_tokens
+    layer = HLTA.for_workload(wl, max_seq_len=n, max_stream_tokens=n)
+    dev = to_device(inp)
+    outs = []
+    for s in range(wl.stream_steps):
+        sl = {k: (v[:, s * n:(s + 1) * n].contiguous() if k != "gates" else v) for k, v in dev.items()}
+        outs.append(layer.stream_step(sl["q"], sl["k"], sl["v"], sl["alpha"], sl["beta"], sl["gates"]))
+    got = to_numpy64(torch.cat(outs, dim=1)).reshape(-1, wl.d_v)
+    S, pos = layer.state_get()
+    torch.cuda.synchronize()
+    assert pos == wl.L
+    rows = sample_rows(wl, n_rows)
+    if heads is None:
+        gdn_out, S_ref = oracle.gdn(inp.q, inp.k, inp.v, inp.alpha, inp.beta)
+        ref = oracle_rows(inp, rows, gdn_out=gdn_out)
+        assert_close(got[rows], ref, wl.dtype, "stream sampled rows")
+        assert_close(to_numpy64(S), S_ref, wl.dtype, "stream final state")
+    else:
+        sub = lambda a: np.ascontiguousarray(a[:, :, heads])
+        gdn_out, S_ref = oracle.gdn(sub(inp.q), sub(inp.k), sub(inp.v), sub(inp.alpha), sub(inp.beta))
+        hs = rows % wl.H
+        keep = np.isin(hs, heads)
+        rows = rows[keep]
+        hmap = {h: i for i, h in enumerate(heads)}
+        bt = rows // wl.H
+        gdn_rows = gdn_out.reshape(-1, len(heads), wl.d_v)[bt, [hmap[h] for h in rows % wl.H]]
+        g = inp.gates.astype(np.float64)[rows % wl.H]
+        ref = oracle_rows(inp, rows, branches=("swa", "dswa")) + g[:, 2, None] * gdn_rows
+        assert_close(got[rows], ref, wl.dtype, "stream sampled rows")
+        assert_close(to_numpy64(S)[:, heads], S_ref, wl.dtype, "stream final state (sampled heads)")
+    layer.close()
+
+
+@pytest.mark.slow
+def test_stream_480p_full_size(torch_cuda):
+    """The streaming workload at full size: B=4, H=24, 120 appends of one
+    1560-token frame; per-step outputs on sampled rows and the final state of
+    sampled heads against the oracle's one-shot pass over 187200 tokens."""
+    _stream_check(torch_cuda, WORKLOADS["stream_480p"], n_rows=1500, heads=[0, 23])
+
+
+def test_stream_checkpoint_resume_bit_identical(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_temporal_b200 import HLTA
+    wl = WORKLOADS["clip_4k"].with_(B=2, H=2, L=8 * 64, P=64, swa_window=70, dswa_window=64,
+                                    dilation=3, stream_steps=8)
+    inp = make_inputs(wl)
+    dev = to_device(inp)
+    n = wl.step_tokens
+    step = lambda layer, s: layer.stream_step(*[dev[k][:, s * n:(s + 1) * n].contiguous()
+                                                for k in ("q", "k", "v", "alpha", "beta")], dev["gates"])
+    a = HLTA.for_workload(wl, max_seq_len=n, max_stream_tokens=n)
+    ref = [step(a, s).clone() for s in range(8)]
+    b = HLTA.for_workload(wl, max_seq_len=n, max_stream_tokens=n)
+    for s in range(4):
+        step(b, s)
+    blob = b.stream_save()
+    c = HLTA.for_workload(wl, max_seq_len=n, max_stream_tokens=n)
+    c.stream_load(blob)
+    for s in range(4, 8):
+        assert torch.equal(step(c, s), ref[s])
+    Sa, pa = a.state_get()
+    Sc, pc = c.state_get()
+    torch.cuda.synchronize()
+    assert pa == pc == wl.L and torch.equal(Sa, Sc)
+    c.stream_reset()
+    assert c.state_get()[1] == 0
+    for x in (a, b, c):
+        x.close()
+
+
+def test_forward_host_matches_device(torch_cuda):
+    wl = WORKLOADS["clip_4k"].with_(H=2, L=512)
+    inp = make_inputs(wl)
+    layer = layer_for(wl)
+    out_dev, _ = run_gpu(layer, to_device(inp))
+    out_host = layer.forward_host(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.gates)
+    np.testing.assert_array_equal(to_numpy64(out_dev),
+                                  (out_host.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    layer.close()
+
+
+def test_rejects_bad_tensors(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_temporal_b200 import HltaError
+    wl = WORKLOADS["clip_4k"].with_(H=2, L=128)
+    layer = layer_for(wl)
+    dev = to_device(make_inputs(wl))
+    lib = layer.lib
+    import ctypes
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    args = [p(dev[k]) for k in ("q", "k", "v", "alpha", "beta", "gates")]
+    out = torch.empty_like(dev["v"])
+    # L beyond max_seq_len, misaligned pointer
+    assert lib.hlta_forward(layer.h, 129, *args, None, None, p(out), 7, None) == 1
+    bad = ctypes.c_void_p(dev["q"].data_ptr() + 2)
+    assert lib.hlta_forward(layer.h, 128, bad, *args[1:], None, None, p(out), 7, None) == 1
+    assert lib.hlta_forward(layer.h, 128, *args, None, None, p(out), 8, None) == 1
+    assert layer.device_status() == 0
+    with pytest.raises(ValueError):
+        layer.forward(dev["q"].float(), dev["k"], dev["v"], dev["alpha"], dev["beta"], dev["gates"])
+    layer.close()

@@ -11,8 +11,11 @@ video of F frames with P tokens each is flattened to a causal sequence of
 L = F * P tokens, token t = f * P + s.  The synthetic workloads stand in for
 latent video; no dataset is involved.
 
-Distributions (all fp64 draws from ``numpy.random.default_rng(seed)``, drawn in
-the order q, k, v, beta, alpha, gates, then cast once):
+Distributions (fp64 draws, cast once).  Every tensor is drawn in blocks of
+4096 tokens per batch element, each block from its own generator
+``default_rng(SeedSequence(seed, spawn_key=(tensor, b, block)))`` with tensor ids
+q=0, k=1, v=2, beta=3, alpha=4, gates=5, so values do not depend on how many
+threads generate them:
 
 * q, k ~ N(0, 1), then L2-normalised per (token, head)
 * v ~ N(0, 1)
@@ -27,15 +30,18 @@ the fp64 draw); ``as_float32`` gives their exact values.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 
 import numpy as np
 
-# Draw block: tensors are generated in blocks of tokens so that the long
-# workloads never hold fp64 copies of the whole tensor.  numpy's Generator
-# continues its stream across calls, so the block size does not change values.
+# Draw block: tensors are generated in independently seeded blocks of tokens,
+# so the long workloads never hold fp64 copies of a whole tensor and blocks can
+# be drawn in parallel.
 _BLOCK_TOKENS = 4096
+_TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "beta": 3, "alpha": 4, "gates": 5}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -86,11 +92,11 @@ ORDER = ["tiny_fp32", "clip_4k", "rollout_480p", "stream_480p", "long_131k"]
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp64/fp32 values to bf16 (nearest, ties to even); return uint16 bits."""
-    f = np.ascontiguousarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    rounding = 0x7FFF + ((u >> 16) & 1)
-    return ((u + rounding) >> 16).astype(np.uint16)
+    """Round fp64/fp32 values to bf16 (nearest, ties to even); return uint16 bits.
+
+    fp64 input is first rounded to fp32 (nearest), then fp32 to bf16."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + (0x7FFF + ((u >> 16) & 1))) >> 16).astype(np.uint16)
 
 
 def bf16_to_float32(bits: np.ndarray) -> np.ndarray:
@@ -117,32 +123,56 @@ class Inputs:
         return bf16_to_float32(a) if a.dtype == np.uint16 else a
 
 
-def _normal_tensor(rng, B, L, H, d, normalise, dtype):
+def _block_rng(seed, tensor, b, block):
+    return np.random.default_rng(np.random.SeedSequence(seed, spawn_key=(_TENSOR_IDS[tensor], b, block)))
+
+
+def _parallel(fn, jobs):
+    workers = min(len(jobs), os.cpu_count() or 1, 16)
+    if workers <= 1:
+        for j in jobs:
+            fn(*j)
+        return
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        list(ex.map(lambda j: fn(*j), jobs))
+
+
+def _normal_tensor(seed, name, B, L, H, d, normalise, dtype):
     out = np.empty((B, L, H, d), dtype=np.uint16 if dtype == "bf16" else np.float32)
+
+    def block(b, blk):
+        t0 = blk * _BLOCK_TOKENS
+        n = min(_BLOCK_TOKENS, L - t0)
+        x = _block_rng(seed, name, b, blk).standard_normal((n, H, d))
+        if normalise:
+            x /= np.linalg.norm(x, axis=-1, keepdims=True)
+        out[b, t0:t0 + n] = bf16_bits(x) if dtype == "bf16" else x.astype(np.float32)
+    _parallel(block, [(b, blk) for b in range(B) for blk in range(-(-L // _BLOCK_TOKENS))])
+    return out
+
+
+def _scalar_tensor(seed, name, B, L, H, fn):
+    out = np.empty((B, L, H), dtype=np.float32)
     for b in range(B):
-        for t0 in range(0, L, _BLOCK_TOKENS):
+        for blk in range(-(-L // _BLOCK_TOKENS)):
+            t0 = blk * _BLOCK_TOKENS
             n = min(_BLOCK_TOKENS, L - t0)
-            x = rng.standard_normal((n, H, d))
-            if normalise:
-                x /= np.linalg.norm(x, axis=-1, keepdims=True)
-            out[b, t0:t0 + n] = bf16_bits(x) if dtype == "bf16" else x.astype(np.float32)
+            out[b, t0:t0 + n] = fn(_block_rng(seed, name, b, blk).standard_normal((n, H)))
     return out
 
 
 def make_inputs(wl: Workload, seed: int | None = None, alpha_mode: str = "default",
                 normalise_qk: bool = True) -> Inputs:
     """Draw the inputs of ``wl`` (see the module docstring for the recipe)."""
-    rng = np.random.default_rng(wl.seed if seed is None else seed)
+    seed = wl.seed if seed is None else seed
     B, L, H = wl.B, wl.L, wl.H
-    q = _normal_tensor(rng, B, L, H, wl.d_k, normalise_qk, wl.dtype)
-    k = _normal_tensor(rng, B, L, H, wl.d_k, normalise_qk, wl.dtype)
-    v = _normal_tensor(rng, B, L, H, wl.d_v, False, wl.dtype)
-    beta = (1.0 / (1.0 + np.exp(-rng.standard_normal((B, L, H))))).astype(np.float32)
+    q = _normal_tensor(seed, "q", B, L, H, wl.d_k, normalise_qk, wl.dtype)
+    k = _normal_tensor(seed, "k", B, L, H, wl.d_k, normalise_qk, wl.dtype)
+    v = _normal_tensor(seed, "v", B, L, H, wl.d_v, False, wl.dtype)
+    beta = _scalar_tensor(seed, "beta", B, L, H, lambda z: 1.0 / (1.0 + np.exp(-z)))
     shift = {"default": wl.alpha_shift, "slow": -4.0}[alpha_mode]
-    z = rng.standard_normal((B, L, H)) + shift
-    softplus = np.logaddexp(0.0, z)
-    alpha = np.exp(-softplus).astype(np.float32)
-    gates = rng.uniform(0.0, 1.0, (H, 3)).astype(np.float32)
+    alpha = _scalar_tensor(seed, "alpha", B, L, H, lambda z: np.exp(-np.logaddexp(0.0, z + shift)))
+    gates = _block_rng(seed, "gates", 0, 0).uniform(0.0, 1.0, (H, 3)).astype(np.float32)
     return Inputs(wl, q, k, v, alpha, beta, gates)
 
 
