@@ -1,5 +1,469 @@
-// tc_attention.cu -- placeholder until the tcgen05 kernel lands.
+// tc_attention.cu -- SWA / DSWA forward on the sm_100a tensor cores (bf16).
+//
+// Kairos paper, section 2.2.2: SWA (Eq. (7), causal window of w keys) and DSWA
+// (Eq. (8): SWA after rearranging frames into residue classes f mod d).
+//
+// Both branches run as one kernel over "segments".  A segment is a run of
+// Pseg consecutive tokens of one (batch, head) sequence: the whole sequence for
+// SWA (Pseg = L), one latent frame for DSWA (Pseg = P).  Segment f of a batch
+// belongs to class g = f mod dil at class position m = f / dil; a token s of it
+// sits at rearranged position r = m*Pseg + s, and query r attends to the keys of
+// its class with r - w < r_k <= r.  SWA is dil = 1 with one segment.  No
+// rearranged copy is made: TMA reads tiles straight from the caller's
+// [B, L, H, d] tensors through a 4-D view (d, H, Pseg, B*F), whose
+// out-of-range rows arrive as zeros.
+//
+// One CTA handles one tile of 128 query rows of one segment (two CTAs per SM):
+//   warp 0      TMA producer: Q once, then K and V tiles (single-buffered)
+//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma
+//                 S = Q K^T   (SS form, 128x128x128, fp32 in TMEM cols 0-127)
+//                 O += P V    (TS form: P read from TMEM, V from smem, MN-major)
+//   warps 2-5   softmax: thread = query row = TMEM lane.  Online softmax in the
+//               log2 domain with a lazily moved reference maximum (O in TMEM is
+//               rescaled only when a row maximum grows by more than 2^8), P is
+//               written back into the S columns as bf16, then the epilogue
+//               scales O by gate/l and writes the row.
+// Key tiles never straddle a segment; tiles crossing the band edge or the
+// segment end are masked per element.
+#include <cuda_bf16.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
 #include "tc_attention.h"
+
 namespace hlta {
-TcAttention *TcAttention::create(const hlta_config &, long long) { return nullptr; }
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;   // query rows per CTA
+constexpr int kBN = 128;   // keys per tile
+constexpr int kD = 128;    // head dim (d_k = d_v)
+constexpr int kMaxKT = 96;
+constexpr int kThreads = 192;
+constexpr uint32_t kTileBytes = kBN * kD * 2;      // 32 KB
+constexpr uint32_t kHalfBytes = kTileBytes / 2;    // one 64-column TMA box
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0;                       // S / P
+constexpr uint32_t kColO = 128;                     // O accumulator
+constexpr float kRescaleThreshold = 8.0f;           // log2 units
+
+struct KeyTile {
+    int seg;     // segment row of the 4-D view: b*Fseg + f
+    int s0;      // first key row inside the segment
+    int rbase;   // rearranged position of that row
+    int kvalid;  // rows of this tile inside the segment
+};
+
+struct TcAttnParams {
+    int Pseg, Fseg, dil, w, tiles_per_seg;
+    int H, L;
+    float scale_log2;
+    const float *gates;
+    int gate_col, out_mode;
+    float *acc;
+    __nv_bfloat16 *out;
+    int *dev_err;
+};
+
+struct __align__(1024) Smem {
+    uint8_t q[kTileBytes];
+    uint8_t k[kTileBytes];
+    uint8_t v[kTileBytes];
+    uint64_t bar_q, bar_k, bar_v, bar_s, bar_p, bar_pv;
+    uint32_t tmem_base;
+    int abort;
+    int nkt;
+    KeyTile kt[kMaxKT];
+};
+
+// Write 32 columns [c0, c0+32) of one output row: out-mode semantics of OutMode.
+__device__ __forceinline__ void store_chunk(const TcAttnParams &p, size_t base, int c0, const uint32_t (&o)[32],
+                                            float scale) {
+    float *acc = p.acc + base + c0;
+    __nv_bfloat16 *out = p.out + base + c0;
+    switch (p.out_mode) {
+        case OUT_STORE:
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+                *reinterpret_cast<float4 *>(acc + c) =
+                    make_float4(__uint_as_float(o[c]) * scale, __uint_as_float(o[c + 1]) * scale,
+                                __uint_as_float(o[c + 2]) * scale, __uint_as_float(o[c + 3]) * scale);
+            break;
+        case OUT_ADD:
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+                float4 a = *reinterpret_cast<float4 *>(acc + c);
+                a.x += __uint_as_float(o[c]) * scale;
+                a.y += __uint_as_float(o[c + 1]) * scale;
+                a.z += __uint_as_float(o[c + 2]) * scale;
+                a.w += __uint_as_float(o[c + 3]) * scale;
+                *reinterpret_cast<float4 *>(acc + c) = a;
+            }
+            break;
+        default: {
+            const bool add = p.out_mode == OUT_FINAL;
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+                float x[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[j] = __uint_as_float(o[c + j]) * scale;
+                if (add) {
+                    const float4 a0 = *reinterpret_cast<const float4 *>(acc + c);
+                    const float4 a1 = *reinterpret_cast<const float4 *>(acc + c + 4);
+                    x[0] += a0.x; x[1] += a0.y; x[2] += a0.z; x[3] += a0.w;
+                    x[4] += a1.x; x[5] += a1.y; x[6] += a1.z; x[7] += a1.w;
+                }
+                uint4 w;
+                w.x = pack_bf16x2(x[0], x[1]);
+                w.y = pack_bf16x2(x[2], x[3]);
+                w.z = pack_bf16x2(x[4], x[5]);
+                w.w = pack_bf16x2(x[6], x[7]);
+                *reinterpret_cast<uint4 *>(out + c) = w;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const TcAttnParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int seg_f = blockIdx.x / p.tiles_per_seg;
+    const int qt = blockIdx.x % p.tiles_per_seg;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int s0 = qt * kBM;
+    const int nq = min(kBM, p.Pseg - s0);
+    const int g = seg_f % p.dil, m = seg_f / p.dil;
+    const int r_min = m * p.Pseg + s0, r_max = r_min + nq - 1;
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        int n = 0;
+        const int lo_r = r_min - p.w + 1;
+        for (int mm = m; mm >= 0; --mm) {
+            const int base = mm * p.Pseg;
+            if (base + p.Pseg - 1 < lo_r) break;
+            const int s_lo = max(0, lo_r - base), s_hi = min(p.Pseg - 1, r_max - base);
+            for (int t = s_lo / kBN; t <= s_hi / kBN && n < kMaxKT; ++t, ++n) {
+                sm.kt[n].seg = b * p.Fseg + g + p.dil * mm;
+                sm.kt[n].s0 = t * kBN;
+                sm.kt[n].rbase = base + t * kBN;
+                sm.kt[n].kvalid = min(kBN, p.Pseg - t * kBN);
+            }
+        }
+        sm.nkt = n;
+        // an earlier launch gave up a wait: do no work (the error stays reported)
+        sm.abort = *reinterpret_cast<volatile int *>(p.dev_err) != 0 ? 1 : 0;
+        mbar_init(&sm.bar_q, 1);
+        mbar_init(&sm.bar_k, 1);
+        mbar_init(&sm.bar_v, 1);
+        mbar_init(&sm.bar_s, 1);
+        mbar_init(&sm.bar_p, 128);
+        mbar_init(&sm.bar_pv, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int nkt = sm.nkt;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            const int qseg = b * p.Fseg + seg_f;
+            mbar_expect_tx(&sm.bar_q, kTileBytes);
+            tma_load_4d(sm.q, &tmQ, 0, h, s0, qseg, &sm.bar_q);
+            tma_load_4d(sm.q + kHalfBytes, &tmQ, 64, h, s0, qseg, &sm.bar_q);
+            int k_issued = 0, v_issued = 0;
+            for (int t = 0; t < nkt; ++t) {
+                const KeyTile kt = sm.kt[t];
+                if (t > 0 && !mbar_wait(&sm.bar_s, (t - 1) & 1, abort, p.dev_err)) break;
+                mbar_expect_tx(&sm.bar_k, kTileBytes);
+                tma_load_4d(sm.k, &tmK, 0, h, kt.s0, kt.seg, &sm.bar_k);
+                tma_load_4d(sm.k + kHalfBytes, &tmK, 64, h, kt.s0, kt.seg, &sm.bar_k);
+                k_issued = t + 1;
+                if (t > 0 && !mbar_wait(&sm.bar_pv, (t - 1) & 1, abort, p.dev_err)) break;
+                mbar_expect_tx(&sm.bar_v, kTileBytes);
+                tma_load_4d(sm.v, &tmV, 0, h, kt.s0, kt.seg, &sm.bar_v);
+                tma_load_4d(sm.v + kHalfBytes, &tmV, 64, h, kt.s0, kt.seg, &sm.bar_v);
+                v_issued = t + 1;
+            }
+            if (*abort) {
+                // let copies in flight land before the CTA's shared memory is released
+                int dummy = 0;
+                volatile int *no_abort = &dummy;
+                mbar_wait(&sm.bar_q, 0, no_abort, nullptr);
+                if (k_issued) mbar_wait(&sm.bar_k, (k_issued - 1) & 1, no_abort, nullptr);
+                if (v_issued) mbar_wait(&sm.bar_v, (v_issued - 1) & 1, no_abort, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+            const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+            const uint32_t qa = smem_u32(sm.q), ka = smem_u32(sm.k), va = smem_u32(sm.v);
+            int committed = 0;
+            if (mbar_wait(&sm.bar_q, 0, abort, p.dev_err)) {
+                for (int t = 0; t < nkt; ++t) {
+                    if (!mbar_wait(&sm.bar_k, t & 1, abort, p.dev_err)) break;
+                    if (t > 0 && !mbar_wait(&sm.bar_pv, (t - 1) & 1, abort, p.dev_err)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
+                        umma_ss(tmem + kColS, smem_desc_sw128(qa + off, 16, 1024),
+                                smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&sm.bar_s);
+                    if (!mbar_wait(&sm.bar_p, t & 1, abort, p.dev_err)) break;
+                    if (!mbar_wait(&sm.bar_v, t & 1, abort, p.dev_err)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        umma_ts(tmem + kColO, tmem + kColS + kk * 8,
+                                smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                                (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&sm.bar_pv);
+                    committed = t + 1;
+                }
+            }
+            if (*abort && committed) {
+                int dummy = 0;
+                volatile int *no_abort = &dummy;
+                mbar_wait(&sm.bar_pv, (committed - 1) & 1, no_abort, nullptr);
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax + epilogue
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const int r_q = r_min + row;
+        float m_ref = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int t = 0; t < nkt && ok; ++t) {
+            // waits are made warp-uniform: the TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_s, t & 1, abort, p.dev_err))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const KeyTile kt = sm.kt[t];
+            const bool full = kt.kvalid == kBN && kt.rbase + kBN - 1 <= r_min && kt.rbase > r_max - p.w;
+            int lo = 0, hi = kBN - 1;
+            if (!full) {
+                lo = max(0, r_q - p.w + 1 - kt.rbase);
+                hi = min(kt.kvalid - 1, r_q - kt.rbase);
+            }
+            // pass 1: row maximum of the scaled, masked scores (32 columns at a time)
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sr[32];
+                tmem_ld32(tl + kColS + c * 32, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int col = c * 32 + j;
+                    const float x = __uint_as_float(sr[j]) * p.scale_log2;
+                    if (full || (col >= lo && col <= hi)) mx = fmaxf(mx, x);
+                }
+            }
+            float scale = 1.f;
+            bool moved = false;
+            if (mx > m_ref + kRescaleThreshold) {
+                scale = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+                m_ref = mx;
+                moved = true;
+            }
+            l_run *= scale;
+            // O holds earlier tiles' contributions from t = 1 on: rescale it
+            if (t > 0 && __any_sync(0xffffffffu, moved)) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_pv, (t - 1) & 1, abort, p.dev_err))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tl + kColO + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * scale);
+                    tmem_st32(tl + kColO + c * 32, o);
+                }
+                tmem_wait_st();
+            }
+            const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+            // pass 2: p = 2^(x - m_ref), written back over S as bf16 pairs
+            float lsum = 0.f;
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                uint32_t sa[32], sb[32], pk[32];
+                tmem_ld32(tl + kColS + hlf * 64, sa);
+                tmem_ld32(tl + kColS + hlf * 64 + 32, sb);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 64; j += 2) {
+                    const int col = hlf * 64 + j;
+                    const uint32_t u0 = j < 32 ? sa[j] : sb[j - 32];
+                    const uint32_t u1 = j < 32 ? sa[j + 1] : sb[j - 31];
+                    float x0 = __uint_as_float(u0) * p.scale_log2 - m_use;
+                    float x1 = __uint_as_float(u1) * p.scale_log2 - m_use;
+                    if (!full && (col < lo || col > hi)) x0 = -INFINITY;
+                    if (!full && (col + 1 < lo || col + 1 > hi)) x1 = -INFINITY;
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    lsum += p0 + p1;
+                    pk[j / 2] = pack_bf16x2(p0, p1);
+                }
+                // P columns [64*hlf, 64*hlf+64) -> TMEM columns [32*hlf, 32*hlf+32); the
+                // S columns they overwrite were read by this or the previous half
+                tmem_st32(tl + kColS + hlf * 32, pk);
+            }
+            l_run += lsum;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_p);
+        }
+        if (ok && nkt > 0 &&
+            __all_sync(0xffffffffu, mbar_wait(&sm.bar_pv, (nkt - 1) & 1, abort, p.dev_err))) {
+            tc_fence_after();
+            const int tok = seg_f * p.Pseg + s0 + row;
+            const size_t base = (((size_t)b * p.L + tok) * p.H + h) * kD;
+            const float scale = p.gates[h * 3 + p.gate_col] / l_run;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tl + kColO + c * 32, r);
+                tmem_wait_ld();
+                if (row < nq) store_chunk(p, base, c * 32, r, scale);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// 4-D view (d, H, Pseg, B*Fseg) of a [B, L, H, d] bf16 tensor, box (64, 1, 128, 1).
+bool make_map(CUtensorMap *map, const void *base, int H, int Pseg, int segs) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)Pseg, (cuuint64_t)segs};
+    const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)Pseg * H * kD * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBN, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+class TcAttentionImpl : public TcAttention {
+public:
+    explicit TcAttentionImpl(const hlta_config &c) : cfg_(c) {}
+
+    cudaError_t run(const void *q, const void *k, const void *v, int L, WindowGeom g, const float *gates,
+                    int gate_col, int mode, float *acc, void *out, int *dev_err, cudaStream_t s,
+                    bool *done) override {
+        *done = false;
+        int Pseg, Fseg;
+        if (g.dil == 1) {
+            Pseg = L;
+            Fseg = 1;
+        } else {
+            if (L % g.P != 0) return cudaSuccess;  // ragged last frame: CUDA-core kernel
+            Pseg = g.P;
+            Fseg = L / g.P;
+        }
+        if (Pseg < kBN) return cudaSuccess;
+        // key tiles one query tile can need: the span w + kBM - 1 rearranged rows,
+        // cut at most at every segment boundary it crosses
+        const long long span = (long long)g.w + kBM - 1;
+        const long long bound = (span + kBN - 1) / kBN + 2 * (span / Pseg + 2);
+        if (bound > kMaxKT) return cudaSuccess;
+        if ((long long)Fseg * Pseg * 1LL > (1LL << 30)) return cudaSuccess;
+
+        CUtensorMap mq, mk, mv;
+        const int segs = cfg_.B * Fseg;
+        if (!make_map(&mq, q, cfg_.H, Pseg, segs) || !make_map(&mk, k, cfg_.H, Pseg, segs) ||
+            !make_map(&mv, v, cfg_.H, Pseg, segs))
+            return cudaErrorInvalidValue;
+        TcAttnParams p;
+        p.Pseg = Pseg;
+        p.Fseg = Fseg;
+        p.dil = g.dil;
+        p.w = g.w;
+        p.tiles_per_seg = (Pseg + kBM - 1) / kBM;
+        p.H = cfg_.H;
+        p.L = L;
+        p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+        p.gates = gates;
+        p.gate_col = gate_col;
+        p.out_mode = mode;
+        p.acc = acc;
+        p.out = static_cast<__nv_bfloat16 *>(out);
+        p.dev_err = dev_err;
+        const size_t smem = sizeof(Smem) + 1024;
+        if (!attr_set_) {
+            cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return e;
+            attr_set_ = true;
+        }
+        const dim3 grid(Fseg * p.tiles_per_seg, cfg_.H, cfg_.B);
+        attn_tc_kernel<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
+        *done = true;
+        return cudaGetLastError();
+    }
+
+private:
+    hlta_config cfg_;
+    bool attr_set_ = false;
+};
+
+}  // namespace
+
+TcAttention *TcAttention::create(const hlta_config &cfg, long long) {
+    if (cfg.dtype != HLTA_BF16 || cfg.d_k != kD || cfg.d_v != kD) return nullptr;
+    return new TcAttentionImpl(cfg);
+}
+
 }  // namespace hlta

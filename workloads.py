@@ -24,6 +24,9 @@ threads generate them:
   workload); ``alpha_mode="slow"`` is a stress variant with shift = -4
   (alpha ~ 0.98) that exercises long memory
 * gates ~ U(0, 1) per head, three per head (SWA, DSWA, GDN)
+* stress variant ``q_scale``: q is multiplied by q_scale after normalising,
+  which sharpens the softmax (logit std ~ 0.0078 * q_scale at d = 128) while
+  the keys stay unit, so the memory stays contractive
 
 bf16 tensors are stored as ``uint16`` bit patterns (round-to-nearest-even of
 the fp64 draw); ``as_float32`` gives their exact values.
@@ -137,7 +140,7 @@ def _parallel(fn, jobs):
         list(ex.map(lambda j: fn(*j), jobs))
 
 
-def _normal_tensor(seed, name, B, L, H, d, normalise, dtype):
+def _normal_tensor(seed, name, B, L, H, d, normalise, dtype, scale=1.0):
     out = np.empty((B, L, H, d), dtype=np.uint16 if dtype == "bf16" else np.float32)
 
     def block(b, blk):
@@ -146,6 +149,8 @@ def _normal_tensor(seed, name, B, L, H, d, normalise, dtype):
         x = _block_rng(seed, name, b, blk).standard_normal((n, H, d))
         if normalise:
             x /= np.linalg.norm(x, axis=-1, keepdims=True)
+        if scale != 1.0:
+            x *= scale
         out[b, t0:t0 + n] = bf16_bits(x) if dtype == "bf16" else x.astype(np.float32)
     _parallel(block, [(b, blk) for b in range(B) for blk in range(-(-L // _BLOCK_TOKENS))])
     return out
@@ -162,11 +167,11 @@ def _scalar_tensor(seed, name, B, L, H, fn):
 
 
 def make_inputs(wl: Workload, seed: int | None = None, alpha_mode: str = "default",
-                normalise_qk: bool = True) -> Inputs:
+                normalise_qk: bool = True, q_scale: float = 1.0) -> Inputs:
     """Draw the inputs of ``wl`` (see the module docstring for the recipe)."""
     seed = wl.seed if seed is None else seed
     B, L, H = wl.B, wl.L, wl.H
-    q = _normal_tensor(seed, "q", B, L, H, wl.d_k, normalise_qk, wl.dtype)
+    q = _normal_tensor(seed, "q", B, L, H, wl.d_k, normalise_qk, wl.dtype, q_scale)
     k = _normal_tensor(seed, "k", B, L, H, wl.d_k, normalise_qk, wl.dtype)
     v = _normal_tensor(seed, "v", B, L, H, wl.d_v, False, wl.dtype)
     beta = _scalar_tensor(seed, "beta", B, L, H, lambda z: 1.0 / (1.0 + np.exp(-z)))
