@@ -2,7 +2,7 @@
 // handle-owned device memory, and the launch sequence of one layer pass.
 //
 // One pass (Kairos paper, section 2.2) runs the selected branches in the order
-// SWA, DSWA, GDN on the caller's stream.  Each branch kernel adds its gated
+// GDN, SWA, DSWA on the caller's stream.  Each branch kernel adds its gated
 // output g[h,b]*o_b into an fp32 accumulator; the last one selected writes the
 // layer output in the configured dtype (fused gate/sum epilogue).
 #include <stdarg.h>
@@ -197,9 +197,12 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
                      float *S_out, void *out, unsigned branches, cudaStream_t s) {
     const hlta_config &c = h->cfg;
     const bool bf16 = c.dtype == HLTA_BF16;
+    // Order: memory first (its per-token column writes only store), then SWA,
+    // then DSWA, whose epilogue reads the accumulator row by row and writes out.
+    const int order[3] = {2, 0, 1};
     int sel[3], n = 0;
-    for (int b = 0; b < 3; ++b)
-        if (branches & (1u << b)) sel[n++] = b;
+    for (int i = 0; i < 3; ++i)
+        if (branches & (1u << order[i])) sel[n++] = order[i];
     if (n == 0) {
         CK(cudaMemsetAsync(out, 0, (size_t)c.B * nq * c.H * c.d_v * h->elem_bytes, s));
         return HLTA_OK;

@@ -13,18 +13,23 @@
 // [B, L, H, d] tensors through a 4-D view (d, H, Pseg, B*F), whose
 // out-of-range rows arrive as zeros.
 //
-// One CTA handles one tile of 128 query rows of one segment (two CTAs per SM):
-//   warp 0      TMA producer: Q once, then K and V tiles (single-buffered)
-//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma
-//                 S = Q K^T   (SS form, 128x128x128, fp32 in TMEM cols 0-127)
-//                 O += P V    (TS form: P read from TMEM, V from smem, MN-major)
-//   warps 2-5   softmax: thread = query row = TMEM lane.  Online softmax in the
-//               log2 domain with a lazily moved reference maximum (O in TMEM is
-//               rescaled only when a row maximum grows by more than 2^8), P is
-//               written back into the S columns as bf16, then the epilogue
-//               scales O by gate/l and writes the row.
-// Key tiles never straddle a segment; tiles crossing the band edge or the
-// segment end are masked per element.
+// One CTA (one per SM) handles two adjacent 128-row query tiles of a segment,
+// which share every K/V tile:
+//   warp 0      TMA producer: Q0, Q1, then K_t and V_t through a 4-slot ring
+//   warp 1      TMEM allocation (512 columns); lane 0 issues tcgen05.mma
+//                 S_j = Q_j K_t^T   (SS form, 128x128x128, fp32 in TMEM)
+//                 O_j += P_j V_t    (TS form: P_j read from TMEM, V_t MN-major)
+//               in the order QK0, QK1, PV0, PV1, so one tile's softmax overlaps
+//               the other tile's MMAs
+//   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: thread = query
+//               row = TMEM lane.  Online softmax in the log2 domain with a
+//               lazily moved reference maximum (O_j is rescaled in TMEM only when
+//               a row maximum grows by more than 2^8); P_j is written back over
+//               S_j as bf16; the epilogue scales O_j by gate/l and writes rows.
+// TMEM: S0 cols 0-127, S1 128-255, O0 256-383, O1 384-511.
+// Key tiles never straddle a segment; a tile is skipped for a query tile whose
+// band it misses, and tiles crossing a band edge or a segment end are masked
+// per element.
 #include <cuda_bf16.h>
 #include <stdio.h>
 
@@ -38,27 +43,27 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128;   // query rows per CTA
+constexpr int kBM = 128;   // rows per query tile
+constexpr int kQT = 2;     // query tiles per CTA
 constexpr int kBN = 128;   // keys per tile
 constexpr int kD = 128;    // head dim (d_k = d_v)
 constexpr int kMaxKT = 96;
-constexpr int kThreads = 192;
-constexpr uint32_t kTileBytes = kBN * kD * 2;      // 32 KB
-constexpr uint32_t kHalfBytes = kTileBytes / 2;    // one 64-column TMA box
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;                       // S / P
-constexpr uint32_t kColO = 128;                     // O accumulator
-constexpr float kRescaleThreshold = 8.0f;           // log2 units
+constexpr int kThreads = 320;
+constexpr int kSlots = 4;                        // K/V ring slots (one 128x128 bf16 tile each)
+constexpr uint32_t kTileBytes = kBN * kD * 2;    // 32 KB
+constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-column TMA box
+constexpr float kRescaleThreshold = 8.0f;        // log2 units
 
 struct KeyTile {
     int seg;     // segment row of the 4-D view: b*Fseg + f
     int s0;      // first key row inside the segment
     int rbase;   // rearranged position of that row
     int kvalid;  // rows of this tile inside the segment
+    uint8_t use[kQT], full[kQT];
 };
 
 struct TcAttnParams {
-    int Pseg, Fseg, dil, w, tiles_per_seg;
+    int Pseg, Fseg, dil, w, qblocks_per_seg;
     int H, L;
     float scale_log2;
     const float *gates;
@@ -69,106 +74,110 @@ struct TcAttnParams {
 };
 
 struct __align__(1024) Smem {
-    uint8_t q[kTileBytes];
-    uint8_t k[kTileBytes];
-    uint8_t v[kTileBytes];
-    uint64_t bar_q, bar_k, bar_v, bar_s, bar_p, bar_pv;
+    uint8_t q[kQT][kTileBytes];
+    uint8_t kv[kSlots][kTileBytes];
+    uint64_t bar_q, full[kSlots], empty[kSlots], bar_s[kQT], bar_p[kQT], bar_pv[kQT];
     uint32_t tmem_base;
     int abort;
     int nkt;
     KeyTile kt[kMaxKT];
 };
 
-// Write 32 columns [c0, c0+32) of one output row: out-mode semantics of OutMode.
+// Write 32 columns [c0, c0+32) of one output row with the OutMode semantics.
+// The accumulator values are all loaded before any store, so the loads overlap
+// instead of waiting on the stores before them.
 __device__ __forceinline__ void store_chunk(const TcAttnParams &p, size_t base, int c0, const uint32_t (&o)[32],
                                             float scale) {
-    float *acc = p.acc + base + c0;
-    __nv_bfloat16 *out = p.out + base + c0;
-    switch (p.out_mode) {
-        case OUT_STORE:
+    float *__restrict__ acc = p.acc + base + c0;
+    __nv_bfloat16 *__restrict__ out = p.out + base + c0;
+    float a[32];
+    if (p.out_mode == OUT_ADD || p.out_mode == OUT_FINAL) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 4)
-                *reinterpret_cast<float4 *>(acc + c) =
-                    make_float4(__uint_as_float(o[c]) * scale, __uint_as_float(o[c + 1]) * scale,
-                                __uint_as_float(o[c + 2]) * scale, __uint_as_float(o[c + 3]) * scale);
-            break;
-        case OUT_ADD:
+        for (int c = 0; c < 32; c += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(acc + c);
+            a[c] = v.x;
+            a[c + 1] = v.y;
+            a[c + 2] = v.z;
+            a[c + 3] = v.w;
+        }
+    } else {
 #pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-                float4 a = *reinterpret_cast<float4 *>(acc + c);
-                a.x += __uint_as_float(o[c]) * scale;
-                a.y += __uint_as_float(o[c + 1]) * scale;
-                a.z += __uint_as_float(o[c + 2]) * scale;
-                a.w += __uint_as_float(o[c + 3]) * scale;
-                *reinterpret_cast<float4 *>(acc + c) = a;
-            }
-            break;
-        default: {
-            const bool add = p.out_mode == OUT_FINAL;
+        for (int c = 0; c < 32; ++c) a[c] = 0.f;
+    }
 #pragma unroll
-            for (int c = 0; c < 32; c += 8) {
-                float x[8];
+    for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(o[c]), scale, a[c]);
+    if (p.out_mode == OUT_STORE || p.out_mode == OUT_ADD) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = __uint_as_float(o[c + j]) * scale;
-                if (add) {
-                    const float4 a0 = *reinterpret_cast<const float4 *>(acc + c);
-                    const float4 a1 = *reinterpret_cast<const float4 *>(acc + c + 4);
-                    x[0] += a0.x; x[1] += a0.y; x[2] += a0.z; x[3] += a0.w;
-                    x[4] += a1.x; x[5] += a1.y; x[6] += a1.z; x[7] += a1.w;
-                }
-                uint4 w;
-                w.x = pack_bf16x2(x[0], x[1]);
-                w.y = pack_bf16x2(x[2], x[3]);
-                w.z = pack_bf16x2(x[4], x[5]);
-                w.w = pack_bf16x2(x[6], x[7]);
-                *reinterpret_cast<uint4 *>(out + c) = w;
-            }
+        for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4 *>(acc + c) = make_float4(a[c], a[c + 1], a[c + 2], a[c + 3]);
+    } else {
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(a[c], a[c + 1]);
+            w.y = pack_bf16x2(a[c + 2], a[c + 3]);
+            w.z = pack_bf16x2(a[c + 4], a[c + 5]);
+            w.w = pack_bf16x2(a[c + 6], a[c + 7]);
+            *reinterpret_cast<uint4 *>(out + c) = w;
         }
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const TcAttnParams p) {
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int seg_f = blockIdx.x / p.tiles_per_seg;
-    const int qt = blockIdx.x % p.tiles_per_seg;
+    const int seg_f = blockIdx.x / p.qblocks_per_seg;
+    const int qb = blockIdx.x % p.qblocks_per_seg;
     const int h = blockIdx.y, b = blockIdx.z;
-    const int s0 = qt * kBM;
-    const int nq = min(kBM, p.Pseg - s0);
+    const int s0 = qb * kQT * kBM;
+    const int nq0 = min(kBM, p.Pseg - s0);
+    const int nq1 = max(0, min(kBM, p.Pseg - s0 - kBM));
     const int g = seg_f % p.dil, m = seg_f / p.dil;
-    const int r_min = m * p.Pseg + s0, r_max = r_min + nq - 1;
+    const int r_min = m * p.Pseg + s0, r_max = r_min + nq0 + nq1 - 1;
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
         int n = 0;
         const int lo_r = r_min - p.w + 1;
+        const int nqs[kQT] = {nq0, nq1};
         for (int mm = m; mm >= 0; --mm) {
             const int base = mm * p.Pseg;
             if (base + p.Pseg - 1 < lo_r) break;
             const int s_lo = max(0, lo_r - base), s_hi = min(p.Pseg - 1, r_max - base);
             for (int t = s_lo / kBN; t <= s_hi / kBN && n < kMaxKT; ++t, ++n) {
-                sm.kt[n].seg = b * p.Fseg + g + p.dil * mm;
-                sm.kt[n].s0 = t * kBN;
-                sm.kt[n].rbase = base + t * kBN;
-                sm.kt[n].kvalid = min(kBN, p.Pseg - t * kBN);
+                KeyTile &k = sm.kt[n];
+                k.seg = b * p.Fseg + g + p.dil * mm;
+                k.s0 = t * kBN;
+                k.rbase = base + t * kBN;
+                k.kvalid = min(kBN, p.Pseg - t * kBN);
+#pragma unroll
+                for (int j = 0; j < kQT; ++j) {
+                    const int lo = r_min + j * kBM, hi = lo + nqs[j] - 1;
+                    k.use[j] = nqs[j] > 0 && k.rbase <= hi && k.rbase + k.kvalid - 1 >= lo - p.w + 1;
+                    k.full[j] = k.kvalid == kBN && k.rbase + kBN - 1 <= lo && k.rbase > hi - p.w;
+                }
             }
         }
         sm.nkt = n;
         // an earlier launch gave up a wait: do no work (the error stays reported)
         sm.abort = *reinterpret_cast<volatile int *>(p.dev_err) != 0 ? 1 : 0;
         mbar_init(&sm.bar_q, 1);
-        mbar_init(&sm.bar_k, 1);
-        mbar_init(&sm.bar_v, 1);
-        mbar_init(&sm.bar_s, 1);
-        mbar_init(&sm.bar_p, 128);
-        mbar_init(&sm.bar_pv, 1);
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], 1);
+        }
+        for (int j = 0; j < kQT; ++j) {
+            mbar_init(&sm.bar_s[j], 1);
+            mbar_init(&sm.bar_p[j], 128);
+            mbar_init(&sm.bar_pv[j], 1);
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -179,108 +188,131 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (lane == 0 && !*abort) {
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
             const int qseg = b * p.Fseg + seg_f;
-            mbar_expect_tx(&sm.bar_q, kTileBytes);
-            tma_load_4d(sm.q, &tmQ, 0, h, s0, qseg, &sm.bar_q);
-            tma_load_4d(sm.q + kHalfBytes, &tmQ, 64, h, s0, qseg, &sm.bar_q);
-            int k_issued = 0, v_issued = 0;
-            for (int t = 0; t < nkt; ++t) {
-                const KeyTile kt = sm.kt[t];
-                if (t > 0 && !mbar_wait(&sm.bar_s, (t - 1) & 1, abort, p.dev_err)) break;
-                mbar_expect_tx(&sm.bar_k, kTileBytes);
-                tma_load_4d(sm.k, &tmK, 0, h, kt.s0, kt.seg, &sm.bar_k);
-                tma_load_4d(sm.k + kHalfBytes, &tmK, 64, h, kt.s0, kt.seg, &sm.bar_k);
-                k_issued = t + 1;
-                if (t > 0 && !mbar_wait(&sm.bar_pv, (t - 1) & 1, abort, p.dev_err)) break;
-                mbar_expect_tx(&sm.bar_v, kTileBytes);
-                tma_load_4d(sm.v, &tmV, 0, h, kt.s0, kt.seg, &sm.bar_v);
-                tma_load_4d(sm.v + kHalfBytes, &tmV, 64, h, kt.s0, kt.seg, &sm.bar_v);
-                v_issued = t + 1;
+            mbar_expect_tx(&sm.bar_q, nq1 > 0 ? 2 * kTileBytes : kTileBytes);
+            for (int j = 0; j < (nq1 > 0 ? 2 : 1); ++j) {
+                tma_load_4d(sm.q[j], &tmQ, 0, h, s0 + j * kBM, qseg, &sm.bar_q);
+                tma_load_4d(sm.q[j] + kHalfBytes, &tmQ, 64, h, s0 + j * kBM, qseg, &sm.bar_q);
+            }
+            int issued = 0;
+            for (int u = 0; u < 2 * nkt; ++u) {
+                const int slot = u % kSlots;
+                if (u >= kSlots && !mbar_wait(&sm.empty[slot], ((u / kSlots) - 1) & 1, abort, p.dev_err)) break;
+                const KeyTile &kt = sm.kt[u >> 1];
+                const CUtensorMap *map = (u & 1) ? &tmV : &tmK;
+                mbar_expect_tx(&sm.full[slot], kTileBytes);
+                tma_load_4d(sm.kv[slot], map, 0, h, kt.s0, kt.seg, &sm.full[slot]);
+                tma_load_4d(sm.kv[slot] + kHalfBytes, map, 64, h, kt.s0, kt.seg, &sm.full[slot]);
+                issued = u + 1;
             }
             if (*abort) {
                 // let copies in flight land before the CTA's shared memory is released
                 int dummy = 0;
                 volatile int *no_abort = &dummy;
                 mbar_wait(&sm.bar_q, 0, no_abort, nullptr);
-                if (k_issued) mbar_wait(&sm.bar_k, (k_issued - 1) & 1, no_abort, nullptr);
-                if (v_issued) mbar_wait(&sm.bar_v, (v_issued - 1) & 1, no_abort, nullptr);
+                for (int u = (issued > kSlots ? issued - kSlots : 0); u < issued; ++u)
+                    mbar_wait(&sm.full[u % kSlots], (u / kSlots) & 1, no_abort, nullptr);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && !*abort) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-            const uint32_t qa = smem_u32(sm.q), ka = smem_u32(sm.k), va = smem_u32(sm.v);
-            int committed = 0;
-            if (mbar_wait(&sm.bar_q, 0, abort, p.dev_err)) {
-                for (int t = 0; t < nkt; ++t) {
-                    if (!mbar_wait(&sm.bar_k, t & 1, abort, p.dev_err)) break;
-                    if (t > 0 && !mbar_wait(&sm.bar_pv, (t - 1) & 1, abort, p.dev_err)) break;
+            int n[kQT] = {0, 0};
+            bool live = mbar_wait(&sm.bar_q, 0, abort, p.dev_err);
+            for (int t = 0; t < nkt && live; ++t) {
+                const KeyTile kt = sm.kt[t];
+                const int uk = 2 * t, uv = 2 * t + 1;
+                const int sk = uk % kSlots, sv = uv % kSlots;
+                if (!(live = mbar_wait(&sm.full[sk], (uk / kSlots) & 1, abort, p.dev_err))) break;
+                const uint32_t ka = smem_u32(sm.kv[sk]);
+#pragma unroll
+                for (int j = 0; j < kQT; ++j) {
+                    if (!kt.use[j]) continue;
+                    if (n[j] > 0 && !(live = mbar_wait(&sm.bar_pv[j], (n[j] - 1) & 1, abort, p.dev_err))) break;
                     tc_fence_after();
+                    const uint32_t qa = smem_u32(sm.q[j]);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk) {
                         const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
-                        umma_ss(tmem + kColS, smem_desc_sw128(qa + off, 16, 1024),
+                        umma_ss(tmem + j * 128, smem_desc_sw128(qa + off, 16, 1024),
                                 smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
                     }
-                    umma_commit(&sm.bar_s);
-                    if (!mbar_wait(&sm.bar_p, t & 1, abort, p.dev_err)) break;
-                    if (!mbar_wait(&sm.bar_v, t & 1, abort, p.dev_err)) break;
+                    umma_commit(&sm.bar_s[j]);
+                }
+                if (!live) break;
+                umma_commit(&sm.empty[sk]);
+                if (!(live = mbar_wait(&sm.full[sv], (uv / kSlots) & 1, abort, p.dev_err))) break;
+                const uint32_t va = smem_u32(sm.kv[sv]);
+#pragma unroll
+                for (int j = 0; j < kQT; ++j) {
+                    if (!kt.use[j]) continue;
+                    if (!(live = mbar_wait(&sm.bar_p[j], n[j] & 1, abort, p.dev_err))) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) {
-                        umma_ts(tmem + kColO, tmem + kColS + kk * 8,
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        umma_ts(tmem + 256 + j * 128, tmem + j * 128 + kk * 8,
                                 smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                                (t > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&sm.bar_pv);
-                    committed = t + 1;
+                                (n[j] > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&sm.bar_pv[j]);
+                    ++n[j];
                 }
+                if (!live) break;
+                umma_commit(&sm.empty[sv]);
             }
-            if (*abort && committed) {
+            if (*abort) {
                 int dummy = 0;
                 volatile int *no_abort = &dummy;
-                mbar_wait(&sm.bar_pv, (committed - 1) & 1, no_abort, nullptr);
+                for (int j = 0; j < kQT; ++j)
+                    if (n[j] > 0) mbar_wait(&sm.bar_pv[j], (n[j] - 1) & 1, no_abort, nullptr);
             }
         }
     } else {
-        // ------------------------------------------------ softmax + epilogue
+        // ------------------------------------------------ softmax + epilogue of tile j
+        const int j = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        const int r_q = r_min + row;
+        const uint32_t colS = j * 128, colO = 256 + j * 128;
+        const int nqj = j == 0 ? nq0 : nq1;
+        const int lo_q = r_min + j * kBM;
+        const int hi_q = lo_q + nqj - 1;
+        const int r_q = lo_q + row;
         float m_ref = -INFINITY, l_run = 0.f;
-        bool ok = true;
+        int n = 0;
+        bool ok = !*abort;
         for (int t = 0; t < nkt && ok; ++t) {
+            const KeyTile &ktr = sm.kt[t];
+            if (!ktr.use[j]) continue;
+            const bool full = ktr.full[j];
+            const int rbase = ktr.rbase, kvalid = ktr.kvalid;
             // waits are made warp-uniform: the TMEM loads below are warp-collective
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_s, t & 1, abort, p.dev_err))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_s[j], n & 1, abort, p.dev_err))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const KeyTile kt = sm.kt[t];
-            const bool full = kt.kvalid == kBN && kt.rbase + kBN - 1 <= r_min && kt.rbase > r_max - p.w;
             int lo = 0, hi = kBN - 1;
             if (!full) {
-                lo = max(0, r_q - p.w + 1 - kt.rbase);
-                hi = min(kt.kvalid - 1, r_q - kt.rbase);
+                lo = max(0, r_q - p.w + 1 - rbase);
+                hi = min(kvalid - 1, r_q - rbase);
             }
             // pass 1: row maximum of the scaled, masked scores (32 columns at a time)
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t sr[32];
-                tmem_ld32(tl + kColS + c * 32, sr);
+                tmem_ld32(tl + colS + c * 32, sr);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int col = c * 32 + j;
-                    const float x = __uint_as_float(sr[j]) * p.scale_log2;
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int col = c * 32 + jj;
+                    const float x = __uint_as_float(sr[jj]) * p.scale_log2;
                     if (full || (col >= lo && col <= hi)) mx = fmaxf(mx, x);
                 }
             }
@@ -292,9 +324,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 moved = true;
             }
             l_run *= scale;
-            // O holds earlier tiles' contributions from t = 1 on: rescale it
-            if (t > 0 && __any_sync(0xffffffffu, moved)) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_pv, (t - 1) & 1, abort, p.dev_err))) {
+            // O_j holds earlier tiles' contributions once n > 0: rescale it
+            if (n > 0 && __any_sync(0xffffffffu, moved)) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_pv[j], (n - 1) & 1, abort, p.dev_err))) {
                     ok = false;
                     break;
                 }
@@ -302,57 +334,58 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
-                    tmem_ld32(tl + kColO + c * 32, o);
+                    tmem_ld32(tl + colO + c * 32, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * scale);
-                    tmem_st32(tl + kColO + c * 32, o);
+                    for (int jj = 0; jj < 32; ++jj) o[jj] = __float_as_uint(__uint_as_float(o[jj]) * scale);
+                    tmem_st32(tl + colO + c * 32, o);
                 }
                 tmem_wait_st();
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            // pass 2: p = 2^(x - m_ref), written back over S as bf16 pairs
+            // pass 2: p = 2^(x - m_ref), written back over S_j as bf16 pairs
             float lsum = 0.f;
 #pragma unroll
             for (int hlf = 0; hlf < 2; ++hlf) {
                 uint32_t sa[32], sb[32], pk[32];
-                tmem_ld32(tl + kColS + hlf * 64, sa);
-                tmem_ld32(tl + kColS + hlf * 64 + 32, sb);
+                tmem_ld32(tl + colS + hlf * 64, sa);
+                tmem_ld32(tl + colS + hlf * 64 + 32, sb);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 64; j += 2) {
-                    const int col = hlf * 64 + j;
-                    const uint32_t u0 = j < 32 ? sa[j] : sb[j - 32];
-                    const uint32_t u1 = j < 32 ? sa[j + 1] : sb[j - 31];
+                for (int jj = 0; jj < 64; jj += 2) {
+                    const int col = hlf * 64 + jj;
+                    const uint32_t u0 = jj < 32 ? sa[jj] : sb[jj - 32];
+                    const uint32_t u1 = jj < 32 ? sa[jj + 1] : sb[jj - 31];
                     float x0 = __uint_as_float(u0) * p.scale_log2 - m_use;
                     float x1 = __uint_as_float(u1) * p.scale_log2 - m_use;
                     if (!full && (col < lo || col > hi)) x0 = -INFINITY;
                     if (!full && (col + 1 < lo || col + 1 > hi)) x1 = -INFINITY;
                     const float p0 = ex2(x0), p1 = ex2(x1);
                     lsum += p0 + p1;
-                    pk[j / 2] = pack_bf16x2(p0, p1);
+                    pk[jj / 2] = pack_bf16x2(p0, p1);
                 }
                 // P columns [64*hlf, 64*hlf+64) -> TMEM columns [32*hlf, 32*hlf+32); the
                 // S columns they overwrite were read by this or the previous half
-                tmem_st32(tl + kColS + hlf * 32, pk);
+                tmem_st32(tl + colS + hlf * 32, pk);
             }
             l_run += lsum;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.bar_p);
+            mbar_arrive(&sm.bar_p[j]);
+            ++n;
         }
-        if (ok && nkt > 0 &&
-            __all_sync(0xffffffffu, mbar_wait(&sm.bar_pv, (nkt - 1) & 1, abort, p.dev_err))) {
+        (void)hi_q;
+        if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.bar_pv[j], (n - 1) & 1, abort, p.dev_err))) {
             tc_fence_after();
-            const int tok = seg_f * p.Pseg + s0 + row;
+            const int tok = seg_f * p.Pseg + s0 + j * kBM + row;
             const size_t base = (((size_t)b * p.L + tok) * p.H + h) * kD;
             const float scale = p.gates[h * 3 + p.gate_col] / l_run;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t r[32];
-                tmem_ld32(tl + kColO + c * 32, r);
+                tmem_ld32(tl + colO + c * 32, r);
                 tmem_wait_ld();
-                if (row < nq) store_chunk(p, base, c * 32, r, scale);
+                if (row < nqj) store_chunk(p, base, c * 32, r, scale);
             }
         }
     }
@@ -361,7 +394,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -416,7 +449,7 @@ public:
         if (Pseg < kBN) return cudaSuccess;
         // key tiles one query tile can need: the span w + kBM - 1 rearranged rows,
         // cut at most at every segment boundary it crosses
-        const long long span = (long long)g.w + kBM - 1;
+        const long long span = (long long)g.w + kQT * kBM - 1;
         const long long bound = (span + kBN - 1) / kBN + 2 * (span / Pseg + 2);
         if (bound > kMaxKT) return cudaSuccess;
         if ((long long)Fseg * Pseg * 1LL > (1LL << 30)) return cudaSuccess;
@@ -431,7 +464,7 @@ public:
         p.Fseg = Fseg;
         p.dil = g.dil;
         p.w = g.w;
-        p.tiles_per_seg = (Pseg + kBM - 1) / kBM;
+        p.qblocks_per_seg = (Pseg + kQT * kBM - 1) / (kQT * kBM);
         p.H = cfg_.H;
         p.L = L;
         p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
@@ -448,7 +481,7 @@ public:
             if (e != cudaSuccess) return e;
             attr_set_ = true;
         }
-        const dim3 grid(Fseg * p.tiles_per_seg, cfg_.H, cfg_.B);
+        const dim3 grid(Fseg * p.qblocks_per_seg, cfg_.H, cfg_.B);
         attn_tc_kernel<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
         *done = true;
         return cudaGetLastError();

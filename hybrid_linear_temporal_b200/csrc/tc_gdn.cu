@@ -1,5 +1,733 @@
-// tc_gdn.cu -- placeholder until the tcgen05 kernel lands.
+// tc_gdn.cu -- chunked gated delta memory on the sm_100a tensor cores (bf16 in).
+//
+// Kairos paper, section 2.2.1: S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T)
+// + beta_t v_t k_t^T and o_t = S_t q_t (retrieval from the decayed state).
+// The recurrence is regrouped into chunks of C = 64 tokens (a derivation, not on
+// the pages).  Inside a chunk with start state S0, l_t = sum_{s<=t} log alpha_s,
+// g_t = exp(l_t) and u_t = beta_t (v_t - alpha_t S_{t-1} k_t):
+//   (I + A) U = diag(beta) V - diag(beta g) K S0^T,  A_ts = beta_t e^{l_t-l_s} k_t.k_s (s < t)
+//   T = (I + A)^-1,  W = T diag(beta g) K,  U~ = T diag(beta) V,  U = U~ - W S0^T
+//   O = diag(g) Q S0^T + Pm U,                Pm_ts = e^{l_t-l_s} q_t.k_s (s <= t)
+//   S_C = g_C S0 + U^T diag(e^{l_C-l}) K.
+// Two kernels:
+//   gdn_prep_kernel  (one CTA per chunk, all chunks in parallel): [K;Q] K^T on
+//       tcgen05 (bf16), the decay masks, T by forward substitution on CUDA cores,
+//       then W^T = K^T (T diag(beta g))^T and U~^T = V^T (T diag(beta))^T as fp16
+//       tcgen05 MMAs.  Writes W and g*Q (fp16), K (fp16), Pm (fp16), U~ (fp32)
+//       and l to a per-chunk scratch.
+//   gdn_scan_kernel  (one CTA per (b, h), chunks in sequence): the d_v = 128 rows
+//       of the state are the MMA's M dimension.  Per chunk:
+//         [S0 W^T | S0 (gQ)^T]  = S16 x [W; gQ]^T      (S16: fp16 copy of S in TMEM)
+//         U^T = U~^T - S0 W^T                         (CUDA cores, fp32)
+//         O^T += U^T Pm^T,  D = (U^T diag(e^{l_C-l})) K   (A operands read from TMEM)
+//         S = g_C S + D  (fp32 in TMEM), S16 = fp16(S), outputs written per token.
+// Internal operands are fp16 (11-bit mantissa) with fp32 accumulation; every
+// value they carry is bounded (unit keys, alpha in (0,1], beta in [0,1]).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
 #include "tc_gdn.h"
+
 namespace hlta {
-TcGdn *TcGdn::create(const hlta_config &, long long) { return nullptr; }
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kC = 64;     // chunk
+constexpr int kD = 128;    // d_k = d_v
+// scratch per chunk
+constexpr size_t kWQBytes = 128 * kD * 2;   // [W; gQ] fp16, 128 rows
+constexpr size_t kK16Bytes = kC * kD * 2;   // K fp16
+constexpr size_t kPmBytes = kC * kC * 2;    // Pm fp16
+constexpr size_t kUtBytes = kC * kD * 4;    // U~ fp32
+constexpr size_t kEllBytes = kC * 4;
+
+struct GdnScratch {
+    __half *wq;   // [BH * NC * 128][128]
+    __half *k16;  // [BH * NC * 64][128]
+    __half *pm;   // [BH * NC * 64][64]
+    float *ut;    // [BH * NC * 64][128]
+    float *ell;   // [BH * NC][64]
+};
+
+// =====================================================================
+// prep
+// =====================================================================
+struct PrepParams {
+    const float *alpha, *beta;  // [B, L, H]
+    int L, H, NC;
+    GdnScratch scr;
+    int *dev_err;
+};
+
+struct __align__(1024) PrepSmem {
+    uint8_t kq[32768];   // 2 regions (d 0-63 / 64-127) x 128 rows: rows 0-63 K, 64-127 Q
+    uint8_t v[16384];    // 2 regions x 64 rows of V
+    uint8_t b1[8192];    // (T diag(beta g))[t][s] fp16, K-major
+    uint8_t b2[8192];    // (T diag(beta))[t][s] fp16
+    float A[kC][kC + 1];
+    float ell[kC], beta[kC], gam[kC];
+    uint64_t bar_tma, bar_mma1, bar_mma2;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk16) {
+    // byte offset of 16-byte chunk `chunk16` (0..7) of row `row` in a 128B-swizzled tile
+    return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(128, 2)
+gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const PrepParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    PrepSmem &sm = *reinterpret_cast<PrepSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const size_t chunk_id = (size_t)bh * p.NC + c;
+    const int t0 = c * kC;
+    volatile int *abort = &sm.abort;
+
+    if (tid == 0) {
+        sm.abort = *reinterpret_cast<volatile int *>(p.dev_err) != 0 ? 1 : 0;
+        mbar_init(&sm.bar_tma, 1);
+        mbar_init(&sm.bar_mma1, 1);
+        mbar_init(&sm.bar_mma2, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+
+    if (tid == 0 && !*abort) {
+        mbar_expect_tx(&sm.bar_tma, 32768 + 16384);
+        tma_load_4d(sm.kq, &tmK, 0, h, t0, b, &sm.bar_tma);
+        tma_load_4d(sm.kq + 8192, &tmQ, 0, h, t0, b, &sm.bar_tma);
+        tma_load_4d(sm.kq + 16384, &tmK, 64, h, t0, b, &sm.bar_tma);
+        tma_load_4d(sm.kq + 24576, &tmQ, 64, h, t0, b, &sm.bar_tma);
+        tma_load_4d(sm.v, &tmV, 0, h, t0, b, &sm.bar_tma);
+        tma_load_4d(sm.v + 8192, &tmV, 64, h, t0, b, &sm.bar_tma);
+    }
+    // decay prefix and beta (tokens past the end act as alpha = 1, beta = 0)
+    if (tid < kC) {
+        const int t = t0 + tid;
+        float la = 0.f, be = 0.f;
+        if (t < p.L) {
+            const size_t i = ((size_t)b * p.L + t) * p.H + h;
+            la = logf(p.alpha[i]);
+            be = p.beta[i];
+        }
+        float x = la;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        sm.ell[tid] = x;  // warp-local prefix; warp 1 adds warp 0's total below
+        sm.beta[tid] = be;
+    }
+    __syncthreads();
+    if (tid >= 32 && tid < kC) sm.ell[tid] += sm.ell[31];
+    __syncthreads();
+    if (tid < kC) {
+        sm.gam[tid] = expf(sm.ell[tid]);
+        p.scr.ell[chunk_id * kC + tid] = sm.ell[tid];
+    }
+
+    // [K; Q] K^T -> TMEM cols 0..63 (bf16 operands, exact products)
+    if (tid == 0) {
+        if (!*abort && mbar_wait(&sm.bar_tma, 0, abort, p.dev_err)) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
+            const uint32_t base = smem_u32(sm.kq);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                umma_ss(tmem, smem_desc_sw128(base + off, 16, 1024), smem_desc_sw128(base + off, 16, 1024),
+                        idesc, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.bar_mma1);
+        }
+    }
+    __syncthreads();  // ell / beta / gam visible
+    const bool ok1 = __all_sync(0xffffffffu, !*abort && mbar_wait(&sm.bar_mma1, 0, abort, p.dev_err));
+    if (ok1) {
+        tc_fence_after();
+        uint32_t g0[32], g1[32];
+        tmem_ld32(tl, g0);
+        tmem_ld32(tl + 32, g1);
+        tmem_wait_ld();
+        if (tid < kC) {
+            const int t = tid;
+            const float lt = sm.ell[t], bt = sm.beta[t];
+#pragma unroll
+            for (int s = 0; s < kC; ++s) {
+                const float gs = __uint_as_float(s < 32 ? g0[s] : g1[s - 32]);
+                sm.A[t][s] = (s < t) ? bt * __expf(lt - sm.ell[s]) * gs : 0.f;
+            }
+        } else {
+            const int t = tid - kC;
+            const float lt = sm.ell[t];
+            uint32_t w[32];
+#pragma unroll
+            for (int s = 0; s < kC; s += 2) {
+                const float q0 = __uint_as_float(s < 32 ? g0[s] : g1[s - 32]);
+                const float q1 = __uint_as_float(s + 1 < 32 ? g0[s + 1] : g1[s + 1 - 32]);
+                const float p0 = (s <= t) ? __expf(lt - sm.ell[s]) * q0 : 0.f;
+                const float p1 = (s + 1 <= t) ? __expf(lt - sm.ell[s + 1]) * q1 : 0.f;
+                w[s / 2] = pack_f16x2(p0, p1);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.scr.pm + (chunk_id * kC + t) * kC);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        }
+    }
+    __syncthreads();
+
+    if (!*abort) {
+        // bf16 -> fp16 in place (Q rows scaled by g_t); K and g*Q copies to the scratch
+        for (int i = tid; i < 2 * 128 * 8; i += 128) {
+            const int region = i >> 10, row = (i >> 3) & 127, ch = i & 7;
+            const uint32_t off = region * 16384 + sw128_off(row, ch);
+            uint4 *ptr = reinterpret_cast<uint4 *>(sm.kq + off);
+            const float scale = row < kC ? 1.f : sm.gam[row - kC];
+            const uint4 f = bf16x8_to_f16x8(*ptr, scale);
+            *ptr = f;
+            const int dcol = region * 64 + ch * 8;
+            if (row < kC)
+                *reinterpret_cast<uint4 *>(p.scr.k16 + (chunk_id * kC + row) * kD + dcol) = f;
+            else
+                *reinterpret_cast<uint4 *>(p.scr.wq + (chunk_id * 128 + row) * kD + dcol) = f;
+        }
+        for (int i = tid; i < 2 * kC * 8; i += 128) {
+            const int region = i >> 9, row = (i >> 3) & 63, ch = i & 7;
+            uint4 *ptr = reinterpret_cast<uint4 *>(sm.v + region * 8192 + sw128_off(row, ch));
+            *ptr = bf16x8_to_f16x8(*ptr, 1.f);
+        }
+        // T = (I + A)^-1 by forward substitution, one column per thread
+        if (tid < kC) {
+            const int j = tid;
+            float Tc[kC];
+#pragma unroll
+            for (int t = 0; t < kC; ++t) {
+                // four partial sums keep the FMA chain of row t short
+                float a0 = (t == j) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                for (int s = 0; s + 3 < t; s += 4) {
+                    a0 = fmaf(-sm.A[t][s], Tc[s], a0);
+                    a1 = fmaf(-sm.A[t][s + 1], Tc[s + 1], a1);
+                    a2 = fmaf(-sm.A[t][s + 2], Tc[s + 2], a2);
+                    a3 = fmaf(-sm.A[t][s + 3], Tc[s + 3], a3);
+                }
+#pragma unroll
+                for (int s = t & ~3; s < t; ++s) a0 = fmaf(-sm.A[t][s], Tc[s], a0);
+                Tc[t] = (a0 + a1) + (a2 + a3);
+            }
+            const float bj = sm.beta[j], bgj = sm.beta[j] * sm.gam[j];
+            __half *b1 = reinterpret_cast<__half *>(sm.b1);
+            __half *b2 = reinterpret_cast<__half *>(sm.b2);
+#pragma unroll
+            for (int t = 0; t < kC; ++t) {
+                const uint32_t off = sw128_off(t, j >> 3) + (j & 7) * 2;
+                b1[off / 2] = __float2half_rn(Tc[t] * bgj);
+                b2[off / 2] = __float2half_rn(Tc[t] * bj);
+            }
+        }
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    // W^T = K^T (T diag(beta g))^T -> cols 64..127; U~^T = V^T (T diag(beta))^T -> cols 128..191
+    if (tid == 0 && !*abort) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f16_f32(128, 64, 1, 0);
+        const uint32_t kb = smem_u32(sm.kq), vb = smem_u32(sm.v);
+        const uint32_t b1 = smem_u32(sm.b1), b2 = smem_u32(sm.b2);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            umma_ss(tmem + 64, smem_desc_sw128(kb + kk * 2048, 16384, 1024), smem_desc_sw128(b1 + kk * 32, 16, 1024),
+                    idesc, kk > 0 ? 1u : 0u);
+            umma_ss(tmem + 128, smem_desc_sw128(vb + kk * 2048, 8192, 1024), smem_desc_sw128(b2 + kk * 32, 16, 1024),
+                    idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.bar_mma2);
+    }
+    const bool ok2 = __all_sync(0xffffffffu, !*abort && mbar_wait(&sm.bar_mma2, 0, abort, p.dev_err));
+    if (ok2) {
+        tc_fence_after();
+        const int r = tid;  // d_k index for W^T, d_v index for U~^T
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t w[32], u[32];
+            tmem_ld32(tl + 64 + half * 32, w);
+            tmem_ld32(tl + 128 + half * 32, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t = half * 32 + j;
+                p.scr.wq[(chunk_id * 128 + t) * kD + r] = __float2half_rn(__uint_as_float(w[j]));
+                p.scr.ut[(chunk_id * kC + t) * kD + r] = __uint_as_float(u[j]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// =====================================================================
+// scan
+// =====================================================================
+struct ScanParams {
+    int L, H, NC;
+    const float *S_in;
+    float *S_out;
+    const float *gates;
+    int out_mode;
+    float *acc;
+    __nv_bfloat16 *out;
+    int *dev_err;
+};
+
+constexpr uint32_t kStageTx = (uint32_t)(kWQBytes + kK16Bytes + kPmBytes + kUtBytes + kEllBytes);
+
+struct __align__(1024) ScanStage {
+    uint8_t wq[kWQBytes];    // 2 regions x 128 rows, K-major SW128
+    uint8_t k16[kK16Bytes];  // 2 regions x 64 rows (d 0-63 / 64-127)
+    uint8_t pm[kPmBytes];    // 64 rows x 64, SW128
+    float ut[kC * kD];       // [t][dv] fp32, unswizzled
+    float ell[kC];
+};
+
+struct __align__(1024) ScanSmem {
+    ScanStage st[2];
+    uint64_t full[2], empty[2], bar_p1, bar_u, bar_o, bar_s16;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// TMEM columns of the scan
+constexpr uint32_t kP1 = 0;     // [S0 W^T | S0 (gQ)^T]  -> O accumulates on cols 64..127
+constexpr uint32_t kU = 128;    // U^T fp16 (32 cols)
+constexpr uint32_t kUd = 160;   // (U^T diag(e^{l_C - l})) fp16
+constexpr uint32_t kS16 = 192;  // fp16 copy of S (64 cols)
+constexpr uint32_t kDS = 256;   // (U^T diag) K
+constexpr uint32_t kSK = 384;   // S fp32
+
+__global__ void __launch_bounds__(192, 1)
+gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant__ CUtensorMap tmK16,
+                const __grid_constant__ CUtensorMap tmPm, const __grid_constant__ CUtensorMap tmUt,
+                const __grid_constant__ CUtensorMap tmEll, const ScanParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    ScanSmem &sm = *reinterpret_cast<ScanSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int bh = b * p.H + h;
+    const int NC = p.NC;
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        sm.abort = *reinterpret_cast<volatile int *>(p.dev_err) != 0 ? 1 : 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], 1 + 128);
+        }
+        mbar_init(&sm.bar_p1, 1);
+        mbar_init(&sm.bar_u, 128);
+        mbar_init(&sm.bar_o, 1);
+        mbar_init(&sm.bar_s16, 128);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmWQ);
+            prefetch_tensormap(&tmK16);
+            prefetch_tensormap(&tmPm);
+            prefetch_tensormap(&tmUt);
+            prefetch_tensormap(&tmEll);
+            int issued = 0;
+            for (int c = 0; c < NC && !*abort; ++c) {
+                const int s = c & 1;
+                if (c >= 2 && !mbar_wait(&sm.empty[s], ((c >> 1) - 1) & 1, abort, p.dev_err)) break;
+                ScanStage &st = sm.st[s];
+                const int cid = bh * NC + c;
+                mbar_expect_tx(&sm.full[s], kStageTx);
+                tma_load_2d(st.wq, &tmWQ, 0, cid * 128, &sm.full[s]);
+                tma_load_2d(st.wq + 16384, &tmWQ, 64, cid * 128, &sm.full[s]);
+                tma_load_2d(st.k16, &tmK16, 0, cid * kC, &sm.full[s]);
+                tma_load_2d(st.k16 + 8192, &tmK16, 64, cid * kC, &sm.full[s]);
+                tma_load_2d(st.pm, &tmPm, 0, cid * kC, &sm.full[s]);
+                tma_load_2d(st.ut, &tmUt, 0, cid * kC, &sm.full[s]);
+                tma_load_2d(st.ell, &tmEll, 0, cid, &sm.full[s]);
+                issued = c + 1;
+            }
+            if (*abort) {
+                int dummy = 0;
+                volatile int *no_abort = &dummy;
+                for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c)
+                    mbar_wait(&sm.full[c & 1], (c >> 1) & 1, no_abort, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id1 = idesc_f16_f32(128, 128, 0, 0);
+            const uint32_t id2 = idesc_f16_f32(128, 64, 0, 0);
+            const uint32_t id3 = idesc_f16_f32(128, 128, 0, 1);
+            int committed = 0;
+            for (int c = 0; c < NC; ++c) {
+                const int s = c & 1;
+                ScanStage &st = sm.st[s];
+                if (!mbar_wait(&sm.full[s], (c >> 1) & 1, abort, p.dev_err)) break;
+                if (!mbar_wait(&sm.bar_s16, c & 1, abort, p.dev_err)) break;
+                tc_fence_after();
+                const uint32_t wq = smem_u32(st.wq);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tmem + kP1, tmem + kS16 + kk * 8,
+                            smem_desc_sw128(wq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id1,
+                            kk > 0 ? 1u : 0u);
+                umma_commit(&sm.bar_p1);
+                if (!mbar_wait(&sm.bar_u, c & 1, abort, p.dev_err)) break;
+                tc_fence_after();
+                const uint32_t pm = smem_u32(st.pm), k16 = smem_u32(st.k16);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    umma_ts(tmem + kP1 + 64, tmem + kU + kk * 8, smem_desc_sw128(pm + kk * 32, 16, 1024), id2, 1u);
+                    umma_ts(tmem + kDS, tmem + kUd + kk * 8, smem_desc_sw128(k16 + kk * 2048, 8192, 1024), id3,
+                            kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sm.bar_o);
+                umma_commit(&sm.empty[s]);
+                committed = c + 1;
+            }
+            if (*abort && committed) {
+                int dummy = 0;
+                volatile int *no_abort = &dummy;
+                mbar_wait(&sm.bar_o, (committed - 1) & 1, no_abort, nullptr);
+            }
+        }
+    } else {
+        // math warps: thread = row of S (d_v index) = TMEM lane
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const float gate = p.gates[h * 3 + 2];
+        // initial state
+        {
+            const float *src = p.S_in ? p.S_in + ((size_t)bh * kD + row) * kD : nullptr;
+            uint32_t f16w[2][32];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t r[32];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    float4 x = src ? *reinterpret_cast<const float4 *>(src + q4 * 32 + j) : make_float4(0, 0, 0, 0);
+                    r[j] = __float_as_uint(x.x);
+                    r[j + 1] = __float_as_uint(x.y);
+                    r[j + 2] = __float_as_uint(x.z);
+                    r[j + 3] = __float_as_uint(x.w);
+                }
+                tmem_st32(tl + kSK + q4 * 32, r);
+#pragma unroll
+                for (int j = 0; j < 32; j += 2)
+                    f16w[q4 >> 1][(q4 & 1) * 16 + j / 2] =
+                        pack_f16x2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+            }
+            tmem_st32(tl + kS16, f16w[0]);
+            tmem_st32(tl + kS16 + 32, f16w[1]);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_s16);
+        }
+        bool ok = true;
+        for (int c = 0; c < NC && ok; ++c) {
+            const int s = c & 1;
+            ScanStage &st = sm.st[s];
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (c >> 1) & 1, abort, p.dev_err) &&
+                                             mbar_wait(&sm.bar_p1, c & 1, abort, p.dev_err))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float lC = st.ell[kC - 1];
+            const float gC = __expf(lC);
+            // U = U~ - S0 W^T  (this row of U^T: 64 tokens)
+            {
+                uint32_t x0[32], x1[32], u[32], ud[32];
+                tmem_ld32(tl + kP1, x0);
+                tmem_ld32(tl + kP1 + 32, x1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int t = 0; t < kC; t += 2) {
+                    const float xa = __uint_as_float(t < 32 ? x0[t] : x1[t - 32]);
+                    const float xb = __uint_as_float(t + 1 < 32 ? x0[t + 1] : x1[t + 1 - 32]);
+                    const float ua = st.ut[t * kD + row] - xa;
+                    const float ub = st.ut[(t + 1) * kD + row] - xb;
+                    u[t / 2] = pack_f16x2(ua, ub);
+                    ud[t / 2] = pack_f16x2(ua * __expf(lC - st.ell[t]), ub * __expf(lC - st.ell[t + 1]));
+                }
+                tmem_st32(tl + kU, u);
+                tmem_st32(tl + kUd, ud);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.bar_u);
+            mbar_arrive(&sm.empty[s]);  // done with this stage's U~ and l
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_o, c & 1, abort, p.dev_err))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tl + kP1 + 64, o0);
+            tmem_ld32(tl + kP1 + 96, o1);
+            // S = g_C S + (U^T diag) K ; S16 = fp16(S)
+            uint32_t f16w[2][32];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t d[32], sk[32];
+                tmem_ld32(tl + kDS + q4 * 32, d);
+                tmem_ld32(tl + kSK + q4 * 32, sk);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    sk[j] = __float_as_uint(fmaf(gC, __uint_as_float(sk[j]), __uint_as_float(d[j])));
+                tmem_st32(tl + kSK + q4 * 32, sk);
+#pragma unroll
+                for (int j = 0; j < 32; j += 2)
+                    f16w[q4 >> 1][(q4 & 1) * 16 + j / 2] =
+                        pack_f16x2(__uint_as_float(sk[j]), __uint_as_float(sk[j + 1]));
+            }
+            tmem_st32(tl + kS16, f16w[0]);
+            tmem_st32(tl + kS16 + 32, f16w[1]);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_s16);
+            // outputs of this chunk (column `row` of 64 output rows); accumulator
+            // values are loaded before any store so the loads overlap
+            const int t0 = c * kC;
+            const size_t stride = (size_t)p.H * kD;
+            const size_t idx0 = (((size_t)b * p.L + t0) * p.H + h) * kD + row;
+            float a[kC];
+#pragma unroll
+            for (int t = 0; t < kC; ++t)
+                a[t] = gate * __uint_as_float(t < 32 ? o0[t] : o1[t - 32]);
+            if (p.out_mode == OUT_ADD || p.out_mode == OUT_FINAL) {
+#pragma unroll
+                for (int t = 0; t < kC; ++t)
+                    if (t0 + t < p.L) a[t] += p.acc[idx0 + t * stride];
+            }
+            if (p.out_mode == OUT_STORE || p.out_mode == OUT_ADD) {
+#pragma unroll
+                for (int t = 0; t < kC; ++t)
+                    if (t0 + t < p.L) p.acc[idx0 + t * stride] = a[t];
+            } else {
+#pragma unroll
+                for (int t = 0; t < kC; ++t)
+                    if (t0 + t < p.L) p.out[idx0 + t * stride] = __float2bfloat16_rn(a[t]);
+            }
+        }
+        if (ok && p.S_out) {
+            tc_fence_after();
+            float *dst = p.S_out + ((size_t)bh * kD + row) * kD;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t r[32];
+                tmem_ld32(tl + kSK + q4 * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(dst + q4 * 32 + j) =
+                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                    __uint_as_float(r[j + 3]));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// =====================================================================
+// host side
+// =====================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+bool map_2d(CUtensorMap *m, CUtensorMapDataType dt, size_t esize, const void *base, uint64_t cols, uint64_t rows,
+            uint32_t box_c, uint32_t box_r, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * esize};
+    const cuuint32_t box[2] = {box_c, box_r};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D view (d, H, L, B) of a [B, L, H, 128] bf16 tensor, box (64, 1, 64, 1).
+bool map_tokens(CUtensorMap *m, const void *base, int H, int L, int B) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)L * H * kD * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+class TcGdnImpl : public TcGdn {
+public:
+    TcGdnImpl(const hlta_config &c, int max_nc) : cfg_(c), max_nc_(max_nc) {}
+    ~TcGdnImpl() override { cudaFree(base_); }
+
+    bool init() {
+        const size_t n = (size_t)cfg_.B * cfg_.H * max_nc_;
+        bytes_ = n * (kWQBytes + kK16Bytes + kPmBytes + kUtBytes + kEllBytes);
+        if (cudaMalloc(&base_, bytes_) != cudaSuccess) {
+            cudaGetLastError();
+            base_ = nullptr;
+            return false;
+        }
+        return true;
+    }
+
+    cudaError_t run(const void *q, const void *k, const void *v, const float *alpha, const float *beta, int L,
+                    const float *S_in, float *S_out, const float *gates, int mode, float *acc, void *out,
+                    int *dev_err, cudaStream_t s, bool *done, int *launches) override {
+        *done = false;
+        if (L < kC) return cudaSuccess;  // shorter than one chunk: recurrent kernel
+        const int NC = (L + kC - 1) / kC;
+        if (NC > max_nc_) return cudaSuccess;
+        const int BH = cfg_.B * cfg_.H;
+        GdnScratch scr;
+        char *p = static_cast<char *>(base_);
+        const size_t n = (size_t)BH * NC;
+        scr.wq = reinterpret_cast<__half *>(p);
+        p += n * kWQBytes;
+        scr.k16 = reinterpret_cast<__half *>(p);
+        p += n * kK16Bytes;
+        scr.pm = reinterpret_cast<__half *>(p);
+        p += n * kPmBytes;
+        scr.ut = reinterpret_cast<float *>(p);
+        p += n * kUtBytes;
+        scr.ell = reinterpret_cast<float *>(p);
+
+        CUtensorMap mq, mk, mv, mwq, mk16, mpm, mut, mell;
+        if (!map_tokens(&mq, q, cfg_.H, L, cfg_.B) || !map_tokens(&mk, k, cfg_.H, L, cfg_.B) ||
+            !map_tokens(&mv, v, cfg_.H, L, cfg_.B) ||
+            !map_2d(&mwq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scr.wq, kD, n * 128, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !map_2d(&mk16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scr.k16, kD, n * kC, 64, kC,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !map_2d(&mpm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scr.pm, kC, n * kC, 64, kC,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !map_2d(&mut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scr.ut, kD, n * kC, kD, kC,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !map_2d(&mell, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scr.ell, kC, n, kC, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+
+        const size_t prep_smem = sizeof(PrepSmem) + 1024, scan_smem = sizeof(ScanSmem) + 1024;
+        if (!attr_set_) {
+            cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)prep_smem);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)scan_smem);
+            if (e != cudaSuccess) return e;
+            attr_set_ = true;
+        }
+        PrepParams pp;
+        pp.alpha = alpha;
+        pp.beta = beta;
+        pp.L = L;
+        pp.H = cfg_.H;
+        pp.NC = NC;
+        pp.scr = scr;
+        pp.dev_err = dev_err;
+        gdn_prep_kernel<<<dim3(NC, cfg_.H, cfg_.B), 128, prep_smem, s>>>(mq, mk, mv, pp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        ScanParams sp;
+        sp.L = L;
+        sp.H = cfg_.H;
+        sp.NC = NC;
+        sp.S_in = S_in;
+        sp.S_out = S_out;
+        sp.gates = gates;
+        sp.out_mode = mode;
+        sp.acc = acc;
+        sp.out = static_cast<__nv_bfloat16 *>(out);
+        sp.dev_err = dev_err;
+        gdn_scan_kernel<<<dim3(cfg_.H, cfg_.B), 192, scan_smem, s>>>(mwq, mk16, mpm, mut, mell, sp);
+        *done = true;
+        if (launches) *launches = 2;
+        return cudaGetLastError();
+    }
+
+private:
+    hlta_config cfg_;
+    int max_nc_;
+    void *base_ = nullptr;
+    size_t bytes_ = 0;
+    bool attr_set_ = false;
+};
+
+}  // namespace
+
+TcGdn *TcGdn::create(const hlta_config &cfg, long long max_seq_len) {
+    if (cfg.dtype != HLTA_BF16 || cfg.d_k != kD || cfg.d_v != kD) return nullptr;
+    long long L = max_seq_len > cfg.max_stream_tokens ? max_seq_len : cfg.max_stream_tokens;
+    const int max_nc = (int)((L + kC - 1) / kC);
+    TcGdnImpl *g = new TcGdnImpl(cfg, max_nc);
+    if (!g->init()) {
+        delete g;
+        return nullptr;
+    }
+    return g;
+}
+
 }  // namespace hlta
