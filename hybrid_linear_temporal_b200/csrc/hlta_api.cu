@@ -82,6 +82,10 @@ struct hlta_handle {
     size_t stage_bytes = 0;
     hlta::TcAttention *tc_attn = nullptr;
     hlta::TcGdn *tc_gdn = nullptr;
+    // concurrent memory branch: side stream, fork/join events, its own accumulator
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    float *acc2 = nullptr;
     // profiling (hlta_profile_enable)
     bool prof = false;
     struct Mark {
@@ -207,6 +211,54 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
         CK(cudaMemsetAsync(out, 0, (size_t)c.B * nq * c.H * c.d_v * h->elem_bytes, s));
         return HLTA_OK;
     }
+    hlta::WindowGeom geo[2];
+    geo[0].P = geo[1].P = c.tokens_per_frame;
+    geo[0].dil = 1;
+    geo[0].w = c.swa_window;
+    geo[1].dil = c.dswa_dilation;
+    geo[1].w = c.dswa_window;
+    const bool want_attn[2] = {(branches & 1u) != 0, (branches & 2u) != 0};
+    // Concurrent schedule: the memory branch (two kernels, one of them a
+    // sequential scan on B*H SMs) runs on the side stream into its own
+    // accumulator while SWA runs on `s`; the last attention branch waits for it
+    // and adds both accumulators in its epilogue.
+    const bool overlap = one_shot && (branches & 4u) && (want_attn[0] || want_attn[1]) && h->side &&
+                         h->acc2 && h->tc_gdn && h->tc_gdn->covers(nq) && h->tc_attn &&
+                         (!want_attn[0] || h->tc_attn->covers(nq, geo[0])) &&
+                         (!want_attn[1] || h->tc_attn->covers(nq, geo[1]));
+    if (overlap) {
+        CK(cudaEventRecord(h->ev_fork, s));
+        CK(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+        {
+            ProfScope ps(h, 2, h->side);
+            bool done = false;
+            int launches = 1;
+            cudaError_t e = h->tc_gdn->run(in.q, in.k, in.v, in.alpha, in.beta, nq, S_in, S_out, in.gates,
+                                           hlta::OUT_STORE, h->acc2, out, h->dev_err, h->side, &done,
+                                           &launches);
+            if (e != cudaSuccess || !done)
+                return fail(HLTA_ERR_CUDA, "tensor-core memory: %s", cudaGetErrorString(e));
+            ps.done(launches);
+        }
+        CK(cudaEventRecord(h->ev_join, h->side));
+        const int na = (int)want_attn[0] + (int)want_attn[1];
+        int idx = 0;
+        for (int br = 0; br < 2; ++br) {
+            if (!want_attn[br]) continue;
+            const bool last = idx == na - 1;
+            if (last) CK(cudaStreamWaitEvent(s, h->ev_join, 0));
+            const int mode = na == 1 ? hlta::OUT_FINAL_ONLY : (last ? hlta::OUT_FINAL : hlta::OUT_STORE);
+            ProfScope ps(h, br, s);
+            bool done = false;
+            cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, geo[br], in.gates, br, mode, h->acc,
+                                            last ? h->acc2 : nullptr, out, h->dev_err, s, &done);
+            if (e != cudaSuccess || !done)
+                return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
+            ps.done(1);
+            ++idx;
+        }
+        return HLTA_OK;
+    }
     for (int idx = 0; idx < n; ++idx) {
         const int br = sel[idx];
         const int mode = out_mode(idx, n);
@@ -220,7 +272,7 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
             bool done = false;
             if (one_shot && h->tc_attn) {
                 cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, g, in.gates, br, mode, h->acc,
-                                                out, h->dev_err, s, &done);
+                                                nullptr, out, h->dev_err, s, &done);
                 if (e != cudaSuccess)
                     return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
             }
@@ -338,6 +390,17 @@ hlta_status hlta_create(const hlta_config *cfg, hlta_handle **out) {
     if (cfg->dtype == HLTA_BF16) {
         h->tc_attn = hlta::TcAttention::create(*cfg, h->acc_rows);
         h->tc_gdn = hlta::TcGdn::create(*cfg, cfg->max_seq_len);
+        if (h->tc_attn && h->tc_gdn) {
+            const size_t acc2_bytes = (size_t)cfg->B * cfg->max_seq_len * cfg->H * cfg->d_v * sizeof(float);
+            if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
+                cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess ||
+                cudaMalloc((void **)&h->acc2, acc2_bytes) != cudaSuccess) {
+                cudaGetLastError();
+                hlta_destroy(h);
+                return fail(HLTA_ERR_OOM, "hlta_create: side stream / accumulator allocation failed");
+            }
+        }
     }
     *out = h;
     return ok();
@@ -353,6 +416,10 @@ hlta_status hlta_destroy(hlta_handle *h) {
     cudaFree(h->ring_k);
     cudaFree(h->ring_v);
     cudaFree(h->stage);
+    cudaFree(h->acc2);
+    if (h->side) cudaStreamDestroy(h->side);
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
     for (auto &m : h->marks) {
         cudaEventDestroy(m.a);
         cudaEventDestroy(m.b);

@@ -47,9 +47,9 @@ constexpr int kBM = 128;   // rows per query tile
 constexpr int kQT = 2;     // query tiles per CTA
 constexpr int kBN = 128;   // keys per tile
 constexpr int kD = 128;    // head dim (d_k = d_v)
-constexpr int kMaxKT = 96;
+constexpr int kMaxKT = 40;
 constexpr int kThreads = 320;
-constexpr int kSlots = 4;                        // K/V ring slots (one 128x128 bf16 tile each)
+constexpr int kSlots = 3;                        // K/V ring slots (one 128x128 bf16 tile each)
 constexpr uint32_t kTileBytes = kBN * kD * 2;    // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-column TMA box
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
@@ -69,13 +69,17 @@ struct TcAttnParams {
     const float *gates;
     int gate_col, out_mode;
     float *acc;
+    const float *acc2;  // optional second accumulator, added in the final modes
     __nv_bfloat16 *out;
     int *dev_err;
 };
 
-struct __align__(1024) Smem {
+// 1024-byte aligned by the kernel (tiles first, each a multiple of 1 KB); the
+// struct itself is not padded to 1 KB so that it fits the 227 KB limit.
+struct __align__(16) Smem {
     uint8_t q[kQT][kTileBytes];
     uint8_t kv[kSlots][kTileBytes];
+    uint8_t pm[kQT][kTileBytes];  // P_j, bf16, K-major 128B-swizzled (A operand of P V)
     uint64_t bar_q, full[kSlots], empty[kSlots], bar_s[kQT], bar_p[kQT], bar_pv[kQT];
     uint32_t tmem_base;
     int abort;
@@ -104,6 +108,17 @@ __device__ __forceinline__ void store_chunk(const TcAttnParams &p, size_t base, 
 #pragma unroll
         for (int c = 0; c < 32; ++c) a[c] = 0.f;
     }
+    if (p.acc2 && (p.out_mode == OUT_FINAL || p.out_mode == OUT_FINAL_ONLY)) {
+        const float *__restrict__ acc2 = p.acc2 + base + c0;
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(acc2 + c);
+            a[c] += v.x;
+            a[c + 1] += v.y;
+            a[c + 2] += v.z;
+            a[c + 3] += v.w;
+        }
+    }
 #pragma unroll
     for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(o[c]), scale, a[c]);
     if (p.out_mode == OUT_STORE || p.out_mode == OUT_ADD) {
@@ -121,6 +136,82 @@ __device__ __forceinline__ void store_chunk(const TcAttnParams &p, size_t base, 
             *reinterpret_cast<uint4 *>(out + c) = w;
         }
     }
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Row maximum of the raw scores in TMEM columns [col, col+128) of this thread's
+// lane.  The softmax scale is positive, so the maximum is taken before scaling.
+// kMask: only columns in [lo, hi] count (band edges, segment ends).
+template <bool kMask>
+__device__ __forceinline__ float tile_row_max(uint32_t taddr, int lo, int hi) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t r[2][32];
+        tmem_ld32(taddr + hlf * 64, r[0]);
+        tmem_ld32(taddr + hlf * 64 + 32, r[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float x0 = __uint_as_float(r[c][j]), x1 = __uint_as_float(r[c][j + 1]);
+                if (kMask) {
+                    const int col = hlf * 64 + c * 32 + j;
+                    if (col < lo || col > hi) x0 = -INFINITY;
+                    if (col + 1 < lo || col + 1 > hi) x1 = -INFINITY;
+                }
+                const int a = (j >> 1) & 7;
+                m[a] = max3f(m[a], x0, x1);
+            }
+    }
+    return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// p = 2^(s*scale - m) over TMEM columns [col, col+128), written as bf16 row
+// `row` of a K-major 128B-swizzled P tile in shared memory (keys 0-63 in the
+// first 16 KB region, keys 64-127 in the second).  Returns the row sum of p.
+template <bool kMask>
+__device__ __forceinline__ float tile_exp_store(uint32_t taddr, float scale, float m, int lo, int hi,
+                                                uint8_t *ptile, int row) {
+    float sum[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sum[i] = 0.f;
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t a[32], b[32], pk[32];
+        tmem_ld32(taddr + hlf * 64, a);
+        tmem_ld32(taddr + hlf * 64 + 32, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) {
+            const uint32_t u0 = j < 32 ? a[j] : b[j - 32];
+            const uint32_t u1 = j < 32 ? a[j + 1] : b[j - 31];
+            float x0 = fmaf(__uint_as_float(u0), scale, -m);
+            float x1 = fmaf(__uint_as_float(u1), scale, -m);
+            if (kMask) {
+                const int col = hlf * 64 + j;
+                if (col < lo || col > hi) x0 = -INFINITY;
+                if (col + 1 < lo || col + 1 > hi) x1 = -INFINITY;
+            }
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            sum[(j >> 1) & 7] += p0 + p1;
+            pk[j >> 1] = pack_bf16x2(p0, p1);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t off = hlf * kHalfBytes + row * 128 + ((c ^ (row & 7)) << 4);
+            *reinterpret_cast<uint4 *>(ptile + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+    }
+    return ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -220,21 +311,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        // Order per key tile t: PV0(t), QK0(t+1), PV1(t), QK1(t+1), so that the
+        // softmax of one query tile runs under the other tile's MMAs.  P_j lives
+        // in shared memory, so S_j may be rewritten as soon as PV_j(t) is issued.
         if (lane == 0 && !*abort) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-            int n[kQT] = {0, 0};
+            int npv[kQT] = {0, 0};
             bool live = mbar_wait(&sm.bar_q, 0, abort, p.dev_err);
-            for (int t = 0; t < nkt && live; ++t) {
-                const KeyTile kt = sm.kt[t];
-                const int uk = 2 * t, uv = 2 * t + 1;
-                const int sk = uk % kSlots, sv = uv % kSlots;
-                if (!(live = mbar_wait(&sm.full[sk], (uk / kSlots) & 1, abort, p.dev_err))) break;
-                const uint32_t ka = smem_u32(sm.kv[sk]);
+            // QK_j for key tile t (K_t must be resident)
+            auto issue_qk = [&](int t) {
+                const uint32_t ka = smem_u32(sm.kv[(2 * t) % kSlots]);
 #pragma unroll
                 for (int j = 0; j < kQT; ++j) {
-                    if (!kt.use[j]) continue;
-                    if (n[j] > 0 && !(live = mbar_wait(&sm.bar_pv[j], (n[j] - 1) & 1, abort, p.dev_err))) break;
+                    if (!sm.kt[t].use[j]) continue;
                     tc_fence_after();
                     const uint32_t qa = smem_u32(sm.q[j]);
 #pragma unroll
@@ -245,31 +335,64 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     }
                     umma_commit(&sm.bar_s[j]);
                 }
-                if (!live) break;
-                umma_commit(&sm.empty[sk]);
+                umma_commit(&sm.empty[(2 * t) % kSlots]);
+            };
+            if (live && nkt > 0) {
+                live = mbar_wait(&sm.full[0], 0, abort, p.dev_err);
+                if (live) issue_qk(0);
+            }
+            for (int t = 0; t < nkt && live; ++t) {
+                const KeyTile kt = sm.kt[t];
+                const int uv = 2 * t + 1, sv = uv % kSlots;
                 if (!(live = mbar_wait(&sm.full[sv], (uv / kSlots) & 1, abort, p.dev_err))) break;
                 const uint32_t va = smem_u32(sm.kv[sv]);
+                const bool more = t + 1 < nkt;
+                bool k_ready = false;
+                uint32_t ka = 0u;
 #pragma unroll
                 for (int j = 0; j < kQT; ++j) {
-                    if (!kt.use[j]) continue;
-                    if (!(live = mbar_wait(&sm.bar_p[j], n[j] & 1, abort, p.dev_err))) break;
-                    tc_fence_after();
+                    if (kt.use[j]) {
+                        if (!(live = mbar_wait(&sm.bar_p[j], npv[j] & 1, abort, p.dev_err))) break;
+                        tc_fence_after();
+                        const uint32_t pa = smem_u32(sm.pm[j]);
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        umma_ts(tmem + 256 + j * 128, tmem + j * 128 + kk * 8,
-                                smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                                (n[j] > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&sm.bar_pv[j]);
-                    ++n[j];
+                        for (int kk = 0; kk < kBN / 16; ++kk) {
+                            const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
+                            umma_ss(tmem + 256 + j * 128, smem_desc_sw128(pa + off, 16, 1024),
+                                    smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                                    (npv[j] > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&sm.bar_pv[j]);
+                        ++npv[j];
+                    }
+                    if (more && sm.kt[t + 1].use[j]) {
+                        if (!k_ready) {
+                            const int uk = 2 * (t + 1);
+                            if (!(live = mbar_wait(&sm.full[uk % kSlots], (uk / kSlots) & 1, abort, p.dev_err)))
+                                break;
+                            ka = smem_u32(sm.kv[uk % kSlots]);
+                            k_ready = true;
+                        }
+                        tc_fence_after();
+                        const uint32_t qa = smem_u32(sm.q[j]);
+#pragma unroll
+                        for (int kk = 0; kk < kD / 16; ++kk) {
+                            const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
+                            umma_ss(tmem + j * 128, smem_desc_sw128(qa + off, 16, 1024),
+                                    smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&sm.bar_s[j]);
+                    }
                 }
                 if (!live) break;
                 umma_commit(&sm.empty[sv]);
+                if (k_ready) umma_commit(&sm.empty[(2 * (t + 1)) % kSlots]);
             }
             if (*abort) {
                 int dummy = 0;
                 volatile int *no_abort = &dummy;
                 for (int j = 0; j < kQT; ++j)
-                    if (n[j] > 0) mbar_wait(&sm.bar_pv[j], (n[j] - 1) & 1, no_abort, nullptr);
+                    if (npv[j] > 0) mbar_wait(&sm.bar_pv[j], (npv[j] - 1) & 1, no_abort, nullptr);
             }
         }
     } else {
@@ -302,20 +425,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 lo = max(0, r_q - p.w + 1 - rbase);
                 hi = min(kvalid - 1, r_q - rbase);
             }
-            // pass 1: row maximum of the scaled, masked scores (32 columns at a time)
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sr[32];
-                tmem_ld32(tl + colS + c * 32, sr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int col = c * 32 + jj;
-                    const float x = __uint_as_float(sr[jj]) * p.scale_log2;
-                    if (full || (col >= lo && col <= hi)) mx = fmaxf(mx, x);
-                }
-            }
+            const float mraw = full ? tile_row_max<false>(tl + colS, lo, hi) : tile_row_max<true>(tl + colS, lo, hi);
+            const float mx = mraw * p.scale_log2;  // -inf stays -inf
             float scale = 1.f;
             bool moved = false;
             if (mx > m_ref + kRescaleThreshold) {
@@ -343,33 +454,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 tmem_wait_st();
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            // pass 2: p = 2^(x - m_ref), written back over S_j as bf16 pairs
-            float lsum = 0.f;
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-                uint32_t sa[32], sb[32], pk[32];
-                tmem_ld32(tl + colS + hlf * 64, sa);
-                tmem_ld32(tl + colS + hlf * 64 + 32, sb);
-                tmem_wait_ld();
-#pragma unroll
-                for (int jj = 0; jj < 64; jj += 2) {
-                    const int col = hlf * 64 + jj;
-                    const uint32_t u0 = jj < 32 ? sa[jj] : sb[jj - 32];
-                    const uint32_t u1 = jj < 32 ? sa[jj + 1] : sb[jj - 31];
-                    float x0 = __uint_as_float(u0) * p.scale_log2 - m_use;
-                    float x1 = __uint_as_float(u1) * p.scale_log2 - m_use;
-                    if (!full && (col < lo || col > hi)) x0 = -INFINITY;
-                    if (!full && (col + 1 < lo || col + 1 > hi)) x1 = -INFINITY;
-                    const float p0 = ex2(x0), p1 = ex2(x1);
-                    lsum += p0 + p1;
-                    pk[jj / 2] = pack_bf16x2(p0, p1);
-                }
-                // P columns [64*hlf, 64*hlf+64) -> TMEM columns [32*hlf, 32*hlf+32); the
-                // S columns they overwrite were read by this or the previous half
-                tmem_st32(tl + colS + hlf * 32, pk);
+            // P_j's buffer is read by PV_j of the previous tile: wait for it (in the
+            // steady state it completed long ago)
+            if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_pv[j], (n - 1) & 1, abort, p.dev_err))) {
+                ok = false;
+                break;
             }
+            const float lsum = full ? tile_exp_store<false>(tl + colS, p.scale_log2, m_use, lo, hi, sm.pm[j], row)
+                                    : tile_exp_store<true>(tl + colS, p.scale_log2, m_use, lo, hi, sm.pm[j], row);
             l_run += lsum;
-            tmem_wait_st();
+            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&sm.bar_p[j]);
             ++n;
@@ -433,26 +527,36 @@ class TcAttentionImpl : public TcAttention {
 public:
     explicit TcAttentionImpl(const hlta_config &c) : cfg_(c) {}
 
+    // Segment geometry of a branch, or false when this kernel does not take it.
+    static bool geometry(int L, WindowGeom g, int *Pseg, int *Fseg) {
+        if (g.dil == 1) {
+            *Pseg = L;
+            *Fseg = 1;
+        } else {
+            if (L % g.P != 0) return false;  // ragged last frame: CUDA-core kernel
+            *Pseg = g.P;
+            *Fseg = L / g.P;
+        }
+        if (*Pseg < kBN) return false;
+        // key tiles one CTA can need: the span w + 2*kBM - 1 rearranged rows, cut
+        // at most at every segment boundary it crosses
+        const long long span = (long long)g.w + kQT * kBM - 1;
+        const long long bound = (span + kBN - 1) / kBN + 2 * (span / *Pseg + 2);
+        if (bound > kMaxKT) return false;
+        return (long long)*Fseg * *Pseg <= (1LL << 30);
+    }
+
+    bool covers(int L, WindowGeom g) const override {
+        int a, b;
+        return geometry(L, g, &a, &b);
+    }
+
     cudaError_t run(const void *q, const void *k, const void *v, int L, WindowGeom g, const float *gates,
-                    int gate_col, int mode, float *acc, void *out, int *dev_err, cudaStream_t s,
-                    bool *done) override {
+                    int gate_col, int mode, float *acc, const float *acc2, void *out, int *dev_err,
+                    cudaStream_t s, bool *done) override {
         *done = false;
         int Pseg, Fseg;
-        if (g.dil == 1) {
-            Pseg = L;
-            Fseg = 1;
-        } else {
-            if (L % g.P != 0) return cudaSuccess;  // ragged last frame: CUDA-core kernel
-            Pseg = g.P;
-            Fseg = L / g.P;
-        }
-        if (Pseg < kBN) return cudaSuccess;
-        // key tiles one query tile can need: the span w + kBM - 1 rearranged rows,
-        // cut at most at every segment boundary it crosses
-        const long long span = (long long)g.w + kQT * kBM - 1;
-        const long long bound = (span + kBN - 1) / kBN + 2 * (span / Pseg + 2);
-        if (bound > kMaxKT) return cudaSuccess;
-        if ((long long)Fseg * Pseg * 1LL > (1LL << 30)) return cudaSuccess;
+        if (!geometry(L, g, &Pseg, &Fseg)) return cudaSuccess;
 
         CUtensorMap mq, mk, mv;
         const int segs = cfg_.B * Fseg;
@@ -472,6 +576,7 @@ public:
         p.gate_col = gate_col;
         p.out_mode = mode;
         p.acc = acc;
+        p.acc2 = acc2;
         p.out = static_cast<__nv_bfloat16 *>(out);
         p.dev_err = dev_err;
         const size_t smem = sizeof(Smem) + 1024;

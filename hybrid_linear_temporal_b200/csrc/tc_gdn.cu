@@ -19,8 +19,9 @@
 //       of the state are the MMA's M dimension.  Per chunk:
 //         [S0 W^T | S0 (gQ)^T]  = S16 x [W; gQ]^T      (S16: fp16 copy of S in TMEM)
 //         U^T = U~^T - S0 W^T                         (CUDA cores, fp32)
-//         O^T += U^T Pm^T,  D = (U^T diag(e^{l_C-l})) K   (A operands read from TMEM)
-//         S = g_C S + D  (fp32 in TMEM), S16 = fp16(S), outputs written per token.
+//         O^T += U^T Pm^T,  D = U^T (diag(e^{l_C-l}) K)   (A operand read from TMEM)
+//         S = g_C S + D  (fp32, held in the math warps' registers), S16 = fp16(S),
+//         outputs written per token.
 // Internal operands are fp16 (11-bit mantissa) with fp32 accumulation; every
 // value they carry is bounded (unit keys, alpha in (0,1], beta in [0,1]).
 #include <cuda_bf16.h>
@@ -43,14 +44,14 @@ constexpr size_t kWQBytes = 128 * kD * 2;   // [W; gQ] fp16, 128 rows
 constexpr size_t kK16Bytes = kC * kD * 2;   // K fp16
 constexpr size_t kPmBytes = kC * kC * 2;    // Pm fp16
 constexpr size_t kUtBytes = kC * kD * 4;    // U~ fp32
-constexpr size_t kEllBytes = kC * 4;
+constexpr size_t kEllBytes = 2 * kC * 4;  // l_t and e^{l_C - l_t}
 
 struct GdnScratch {
     __half *wq;   // [BH * NC * 128][128]
-    __half *k16;  // [BH * NC * 64][128]
+    __half *k16;  // [BH * NC * 64][128]: e^{l_C - l_t} k_t
     __half *pm;   // [BH * NC * 64][64]
     float *ut;    // [BH * NC * 64][128]
-    float *ell;   // [BH * NC][64]
+    float *ell;   // [BH * NC][128]: l_t, then e^{l_C - l_t}
 };
 
 // =====================================================================
@@ -59,6 +60,7 @@ struct GdnScratch {
 struct PrepParams {
     const float *alpha, *beta;  // [B, L, H]
     int L, H, NC;
+    int c_begin;                // first chunk of this launch (blockIdx.x is relative)
     GdnScratch scr;
     int *dev_err;
 };
@@ -68,8 +70,8 @@ struct __align__(1024) PrepSmem {
     uint8_t v[16384];    // 2 regions x 64 rows of V
     uint8_t b1[8192];    // (T diag(beta g))[t][s] fp16, K-major
     uint8_t b2[8192];    // (T diag(beta))[t][s] fp16
-    float A[kC][kC + 1];
-    float ell[kC], beta[kC], gam[kC];
+    float A[kC][kC + 4];  // rows padded to 16 bytes
+    float ell[kC], beta[kC], gam[kC], dec[kC];
     uint64_t bar_tma, bar_mma1, bar_mma2;
     uint32_t tmem_base;
     int abort;
@@ -86,7 +88,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     PrepSmem &sm = *reinterpret_cast<PrepSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int c = p.c_begin + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
     const size_t chunk_id = (size_t)bh * p.NC + c;
     const int t0 = c * kC;
@@ -141,7 +143,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
     if (tid < kC) {
         sm.gam[tid] = expf(sm.ell[tid]);
-        p.scr.ell[chunk_id * kC + tid] = sm.ell[tid];
+        sm.dec[tid] = expf(sm.ell[kC - 1] - sm.ell[tid]);
+        p.scr.ell[chunk_id * 2 * kC + tid] = sm.ell[tid];
+        p.scr.ell[chunk_id * 2 * kC + kC + tid] = sm.dec[tid];
     }
 
     // [K; Q] K^T -> TMEM cols 0..63 (bf16 operands, exact products)
@@ -171,9 +175,14 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int t = tid;
             const float lt = sm.ell[t], bt = sm.beta[t];
 #pragma unroll
-            for (int s = 0; s < kC; ++s) {
-                const float gs = __uint_as_float(s < 32 ? g0[s] : g1[s - 32]);
-                sm.A[t][s] = (s < t) ? bt * __expf(lt - sm.ell[s]) * gs : 0.f;
+            for (int s = 0; s < kC; s += 4) {
+                float a[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float gs = __uint_as_float(s + e < 32 ? g0[s + e] : g1[s + e - 32]);
+                    a[e] = (s + e < t) ? bt * __expf(lt - sm.ell[s + e]) * gs : 0.f;
+                }
+                *reinterpret_cast<float4 *>(&sm.A[t][s]) = make_float4(a[0], a[1], a[2], a[3]);
             }
         } else {
             const int t = tid - kC;
@@ -195,42 +204,47 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
 
     if (!*abort) {
-        // bf16 -> fp16 in place (Q rows scaled by g_t); K and g*Q copies to the scratch
-        for (int i = tid; i < 2 * 128 * 8; i += 128) {
-            const int region = i >> 10, row = (i >> 3) & 127, ch = i & 7;
-            const uint32_t off = region * 16384 + sw128_off(row, ch);
-            uint4 *ptr = reinterpret_cast<uint4 *>(sm.kq + off);
-            const float scale = row < kC ? 1.f : sm.gam[row - kC];
-            const uint4 f = bf16x8_to_f16x8(*ptr, scale);
-            *ptr = f;
-            const int dcol = region * 64 + ch * 8;
-            if (row < kC)
-                *reinterpret_cast<uint4 *>(p.scr.k16 + (chunk_id * kC + row) * kD + dcol) = f;
-            else
-                *reinterpret_cast<uint4 *>(p.scr.wq + (chunk_id * 128 + row) * kD + dcol) = f;
-        }
-        for (int i = tid; i < 2 * kC * 8; i += 128) {
-            const int region = i >> 9, row = (i >> 3) & 63, ch = i & 7;
-            uint4 *ptr = reinterpret_cast<uint4 *>(sm.v + region * 8192 + sw128_off(row, ch));
-            *ptr = bf16x8_to_f16x8(*ptr, 1.f);
-        }
-        // T = (I + A)^-1 by forward substitution, one column per thread
-        if (tid < kC) {
+        if (tid >= kC) {
+            // threads 64..127, while 0..63 solve: bf16 -> fp16 in place (Q rows scaled
+            // by g_t), and the K and g*Q copies to the scratch
+            for (int i = tid - kC; i < 2 * 128 * 8; i += kC) {
+                const int region = i >> 10, row = (i >> 3) & 127, ch = i & 7;
+                const uint32_t off = region * 16384 + sw128_off(row, ch);
+                uint4 *ptr = reinterpret_cast<uint4 *>(sm.kq + off);
+                const uint4 raw = *ptr;
+                const uint4 f = bf16x8_to_f16x8(raw, row < kC ? 1.f : sm.gam[row - kC]);
+                *ptr = f;
+                const int dcol = region * 64 + ch * 8;
+                if (row < kC)  // the scan's copy of K carries the decay to the chunk end
+                    *reinterpret_cast<uint4 *>(p.scr.k16 + (chunk_id * kC + row) * kD + dcol) =
+                        bf16x8_to_f16x8(raw, sm.dec[row]);
+                else
+                    *reinterpret_cast<uint4 *>(p.scr.wq + (chunk_id * 128 + row) * kD + dcol) = f;
+            }
+            for (int i = tid - kC; i < 2 * kC * 8; i += kC) {
+                const int region = i >> 9, row = (i >> 3) & 63, ch = i & 7;
+                uint4 *ptr = reinterpret_cast<uint4 *>(sm.v + region * 8192 + sw128_off(row, ch));
+                *ptr = bf16x8_to_f16x8(*ptr, 1.f);
+            }
+        } else {
+            // T = (I + A)^-1 by forward substitution, one column per thread.  Row t
+            // of A is zero from column t on and the not-yet-computed entries of the
+            // column are zero, so whole 4-column groups can be read.
             const int j = tid;
             float Tc[kC];
 #pragma unroll
+            for (int t = 0; t < kC; ++t) Tc[t] = 0.f;
+#pragma unroll
             for (int t = 0; t < kC; ++t) {
-                // four partial sums keep the FMA chain of row t short
                 float a0 = (t == j) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                for (int s = 0; s + 3 < t; s += 4) {
-                    a0 = fmaf(-sm.A[t][s], Tc[s], a0);
-                    a1 = fmaf(-sm.A[t][s + 1], Tc[s + 1], a1);
-                    a2 = fmaf(-sm.A[t][s + 2], Tc[s + 2], a2);
-                    a3 = fmaf(-sm.A[t][s + 3], Tc[s + 3], a3);
+                for (int g4 = 0; g4 < (t + 3) / 4; ++g4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(&sm.A[t][4 * g4]);
+                    a0 = fmaf(-a4.x, Tc[4 * g4], a0);
+                    a1 = fmaf(-a4.y, Tc[4 * g4 + 1], a1);
+                    a2 = fmaf(-a4.z, Tc[4 * g4 + 2], a2);
+                    a3 = fmaf(-a4.w, Tc[4 * g4 + 3], a3);
                 }
-#pragma unroll
-                for (int s = t & ~3; s < t; ++s) a0 = fmaf(-sm.A[t][s], Tc[s], a0);
                 Tc[t] = (a0 + a1) + (a2 + a3);
             }
             const float bj = sm.beta[j], bgj = sm.beta[j] * sm.gam[j];
@@ -293,6 +307,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 // =====================================================================
 struct ScanParams {
     int L, H, NC;
+    int c_begin, nseg;  // this launch scans chunks [c_begin, c_begin + nseg)
     const float *S_in;
     float *S_out;
     const float *gates;
@@ -309,7 +324,7 @@ struct __align__(1024) ScanStage {
     uint8_t k16[kK16Bytes];  // 2 regions x 64 rows (d 0-63 / 64-127)
     uint8_t pm[kPmBytes];    // 64 rows x 64, SW128
     float ut[kC * kD];       // [t][dv] fp32, unswizzled
-    float ell[kC];
+    float ell[2 * kC];       // l_t, then e^{l_C - l_t}
 };
 
 struct __align__(1024) ScanSmem {
@@ -322,12 +337,12 @@ struct __align__(1024) ScanSmem {
 // TMEM columns of the scan
 constexpr uint32_t kP1 = 0;     // [S0 W^T | S0 (gQ)^T]  -> O accumulates on cols 64..127
 constexpr uint32_t kU = 128;    // U^T fp16 (32 cols)
-constexpr uint32_t kUd = 160;   // (U^T diag(e^{l_C - l})) fp16
 constexpr uint32_t kS16 = 192;  // fp16 copy of S (64 cols)
-constexpr uint32_t kDS = 256;   // (U^T diag) K
-constexpr uint32_t kSK = 384;   // S fp32
+constexpr uint32_t kDS = 256;   // U^T (diag(e^{l_C - l}) K)
 
-__global__ void __launch_bounds__(192, 1)
+constexpr int kScanThreads = 320;  // producer, MMA issuer, 8 math warps
+
+__global__ void __launch_bounds__(kScanThreads, 1)
 gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant__ CUtensorMap tmK16,
                 const __grid_constant__ CUtensorMap tmPm, const __grid_constant__ CUtensorMap tmUt,
                 const __grid_constant__ CUtensorMap tmEll, const ScanParams p) {
@@ -336,19 +351,19 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x, b = blockIdx.y;
     const int bh = b * p.H + h;
-    const int NC = p.NC;
+    const int NC = p.nseg;  // chunks of this launch; chunk c here is p.c_begin + c
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
         sm.abort = *reinterpret_cast<volatile int *>(p.dev_err) != 0 ? 1 : 0;
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], 1 + 128);
+            mbar_init(&sm.empty[i], 1 + 256);
         }
         mbar_init(&sm.bar_p1, 1);
-        mbar_init(&sm.bar_u, 128);
+        mbar_init(&sm.bar_u, 256);
         mbar_init(&sm.bar_o, 1);
-        mbar_init(&sm.bar_s16, 128);
+        mbar_init(&sm.bar_s16, 256);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -372,7 +387,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
                 const int s = c & 1;
                 if (c >= 2 && !mbar_wait(&sm.empty[s], ((c >> 1) - 1) & 1, abort, p.dev_err)) break;
                 ScanStage &st = sm.st[s];
-                const int cid = bh * NC + c;
+                const int cid = bh * p.NC + p.c_begin + c;
                 mbar_expect_tx(&sm.full[s], kStageTx);
                 tma_load_2d(st.wq, &tmWQ, 0, cid * 128, &sm.full[s]);
                 tma_load_2d(st.wq + 16384, &tmWQ, 64, cid * 128, &sm.full[s]);
@@ -415,7 +430,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     umma_ts(tmem + kP1 + 64, tmem + kU + kk * 8, smem_desc_sw128(pm + kk * 32, 16, 1024), id2, 1u);
-                    umma_ts(tmem + kDS, tmem + kUd + kk * 8, smem_desc_sw128(k16 + kk * 2048, 8192, 1024), id3,
+                    umma_ts(tmem + kDS, tmem + kU + kk * 8, smem_desc_sw128(k16 + kk * 2048, 8192, 1024), id3,
                             kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&sm.bar_o);
@@ -429,34 +444,29 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
             }
         }
     } else {
-        // math warps: thread = row of S (d_v index) = TMEM lane
+        // math warps: two groups of four; thread = row of S (d_v index) = TMEM lane.
+        // Group w takes tokens [32w, 32w+32) of U and O and d_k columns
+        // [64w, 64w+64) of the state, which it keeps in fp32 registers.
+        const int w = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const float gate = p.gates[h * 3 + 2];
-        // initial state
+        float S[64];
         {
-            const float *src = p.S_in ? p.S_in + ((size_t)bh * kD + row) * kD : nullptr;
-            uint32_t f16w[2][32];
+            const float *src = p.S_in ? p.S_in + ((size_t)bh * kD + row) * kD + 64 * w : nullptr;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t r[32];
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    float4 x = src ? *reinterpret_cast<const float4 *>(src + q4 * 32 + j) : make_float4(0, 0, 0, 0);
-                    r[j] = __float_as_uint(x.x);
-                    r[j + 1] = __float_as_uint(x.y);
-                    r[j + 2] = __float_as_uint(x.z);
-                    r[j + 3] = __float_as_uint(x.w);
-                }
-                tmem_st32(tl + kSK + q4 * 32, r);
-#pragma unroll
-                for (int j = 0; j < 32; j += 2)
-                    f16w[q4 >> 1][(q4 & 1) * 16 + j / 2] =
-                        pack_f16x2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+            for (int j = 0; j < 64; j += 4) {
+                const float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
+                S[j] = x.x;
+                S[j + 1] = x.y;
+                S[j + 2] = x.z;
+                S[j + 3] = x.w;
             }
-            tmem_st32(tl + kS16, f16w[0]);
-            tmem_st32(tl + kS16 + 32, f16w[1]);
+            uint32_t f16w[32];
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) f16w[j / 2] = pack_f16x2(S[j], S[j + 1]);
+            tmem_st32(tl + kS16 + 32 * w, f16w);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.bar_s16);
@@ -471,25 +481,19 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
                 break;
             }
             tc_fence_after();
-            const float lC = st.ell[kC - 1];
-            const float gC = __expf(lC);
-            // U = U~ - S0 W^T  (this row of U^T: 64 tokens)
+            const float gC = __expf(st.ell[kC - 1]);
+            // U = U~ - S0 W^T for tokens [32w, 32w+32) of this row of U^T
             {
-                uint32_t x0[32], x1[32], u[32], ud[32];
-                tmem_ld32(tl + kP1, x0);
-                tmem_ld32(tl + kP1 + 32, x1);
+                uint32_t x[32], u[16];
+                tmem_ld32(tl + kP1 + 32 * w, x);
                 tmem_wait_ld();
 #pragma unroll
-                for (int t = 0; t < kC; t += 2) {
-                    const float xa = __uint_as_float(t < 32 ? x0[t] : x1[t - 32]);
-                    const float xb = __uint_as_float(t + 1 < 32 ? x0[t + 1] : x1[t + 1 - 32]);
-                    const float ua = st.ut[t * kD + row] - xa;
-                    const float ub = st.ut[(t + 1) * kD + row] - xb;
-                    u[t / 2] = pack_f16x2(ua, ub);
-                    ud[t / 2] = pack_f16x2(ua * __expf(lC - st.ell[t]), ub * __expf(lC - st.ell[t + 1]));
+                for (int j = 0; j < 32; j += 2) {
+                    const int t = 32 * w + j;
+                    u[j / 2] = pack_f16x2(st.ut[t * kD + row] - __uint_as_float(x[j]),
+                                          st.ut[(t + 1) * kD + row] - __uint_as_float(x[j + 1]));
                 }
-                tmem_st32(tl + kU, u);
-                tmem_st32(tl + kUd, ud);
+                tmem_st16(tl + kU + 16 * w, u);
                 tmem_wait_st();
             }
             tc_fence_before();
@@ -500,69 +504,62 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
                 break;
             }
             tc_fence_after();
-            uint32_t o0[32], o1[32];
-            tmem_ld32(tl + kP1 + 64, o0);
-            tmem_ld32(tl + kP1 + 96, o1);
-            // S = g_C S + (U^T diag) K ; S16 = fp16(S)
-            uint32_t f16w[2][32];
+            // S = g_C S + U^T (diag(e^{l_C - l}) K) on columns [64w, 64w+64); S16 = fp16(S)
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t d[32], sk[32];
-                tmem_ld32(tl + kDS + q4 * 32, d);
-                tmem_ld32(tl + kSK + q4 * 32, sk);
+            for (int q2 = 0; q2 < 2; ++q2) {
+                uint32_t d[32], f16w[16];
+                tmem_ld32(tl + kDS + 64 * w + 32 * q2, d);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    sk[j] = __float_as_uint(fmaf(gC, __uint_as_float(sk[j]), __uint_as_float(d[j])));
-                tmem_st32(tl + kSK + q4 * 32, sk);
-#pragma unroll
-                for (int j = 0; j < 32; j += 2)
-                    f16w[q4 >> 1][(q4 & 1) * 16 + j / 2] =
-                        pack_f16x2(__uint_as_float(sk[j]), __uint_as_float(sk[j + 1]));
+                for (int j = 0; j < 32; j += 2) {
+                    float &s0 = S[32 * q2 + j], &s1 = S[32 * q2 + j + 1];
+                    s0 = fmaf(gC, s0, __uint_as_float(d[j]));
+                    s1 = fmaf(gC, s1, __uint_as_float(d[j + 1]));
+                    f16w[j / 2] = pack_f16x2(s0, s1);
+                }
+                tmem_st16(tl + kS16 + 32 * w + 16 * q2, f16w);
             }
-            tmem_st32(tl + kS16, f16w[0]);
-            tmem_st32(tl + kS16 + 32, f16w[1]);
+            // O for tokens [32w, 32w+32) must be read before the next chunk's MMA
+            // overwrites it, i.e. before S16 is released
+            uint32_t o[32];
+            tmem_ld32(tl + kP1 + 64 + 32 * w, o);
+            tmem_wait_ld();
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.bar_s16);
-            // outputs of this chunk (column `row` of 64 output rows); accumulator
-            // values are loaded before any store so the loads overlap
-            const int t0 = c * kC;
+            // outputs of tokens [32w, 32w+32) of this chunk, column `row`, in groups
+            // of 8 tokens whose accumulator loads are issued before their stores
+            const int t0 = (p.c_begin + c) * kC + 32 * w;
+            const int nt = min(32, p.L - t0);
             const size_t stride = (size_t)p.H * kD;
             const size_t idx0 = (((size_t)b * p.L + t0) * p.H + h) * kD + row;
-            float a[kC];
+            const bool add = p.out_mode == OUT_ADD || p.out_mode == OUT_FINAL;
+            const bool to_acc = p.out_mode == OUT_STORE || p.out_mode == OUT_ADD;
 #pragma unroll
-            for (int t = 0; t < kC; ++t)
-                a[t] = gate * __uint_as_float(t < 32 ? o0[t] : o1[t - 32]);
-            if (p.out_mode == OUT_ADD || p.out_mode == OUT_FINAL) {
+            for (int g8 = 0; g8 < 4; ++g8) {
+                float v8[8];
 #pragma unroll
-                for (int t = 0; t < kC; ++t)
-                    if (t0 + t < p.L) a[t] += p.acc[idx0 + t * stride];
-            }
-            if (p.out_mode == OUT_STORE || p.out_mode == OUT_ADD) {
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 8 * g8 + e;
+                    v8[e] = gate * __uint_as_float(o[t]);
+                    if (add && t < nt) v8[e] += p.acc[idx0 + t * stride];
+                }
 #pragma unroll
-                for (int t = 0; t < kC; ++t)
-                    if (t0 + t < p.L) p.acc[idx0 + t * stride] = a[t];
-            } else {
-#pragma unroll
-                for (int t = 0; t < kC; ++t)
-                    if (t0 + t < p.L) p.out[idx0 + t * stride] = __float2bfloat16_rn(a[t]);
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 8 * g8 + e;
+                    if (t >= nt) continue;
+                    if (to_acc)
+                        p.acc[idx0 + t * stride] = v8[e];
+                    else
+                        p.out[idx0 + t * stride] = __float2bfloat16_rn(v8[e]);
+                }
             }
         }
         if (ok && p.S_out) {
-            tc_fence_after();
-            float *dst = p.S_out + ((size_t)bh * kD + row) * kD;
+            float *dst = p.S_out + ((size_t)bh * kD + row) * kD + 64 * w;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t r[32];
-                tmem_ld32(tl + kSK + q4 * 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(dst + q4 * 32 + j) =
-                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                    __uint_as_float(r[j + 3]));
-            }
+            for (int j = 0; j < 64; j += 4)
+                *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     }
 
@@ -622,18 +619,25 @@ bool map_tokens(CUtensorMap *m, const void *base, int H, int L, int B) {
 class TcGdnImpl : public TcGdn {
 public:
     TcGdnImpl(const hlta_config &c, int max_nc) : cfg_(c), max_nc_(max_nc) {}
-    ~TcGdnImpl() override { cudaFree(base_); }
+    ~TcGdnImpl() override {
+        cudaFree(base_);
+        cudaFree(s_mid_);
+        if (prep_stream_) cudaStreamDestroy(prep_stream_);
+        for (auto e : ev_) if (e) cudaEventDestroy(e);
+    }
 
     bool init() {
         const size_t n = (size_t)cfg_.B * cfg_.H * max_nc_;
         bytes_ = n * (kWQBytes + kK16Bytes + kPmBytes + kUtBytes + kEllBytes);
-        if (cudaMalloc(&base_, bytes_) != cudaSuccess) {
-            cudaGetLastError();
-            base_ = nullptr;
-            return false;
-        }
-        return true;
+        const size_t sbytes = (size_t)cfg_.B * cfg_.H * kD * kD * sizeof(float);
+        bool ok = cudaMalloc(&base_, bytes_) == cudaSuccess && cudaMalloc(&s_mid_, 2 * sbytes) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&prep_stream_, cudaStreamNonBlocking) == cudaSuccess;
+        for (auto &e : ev_) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) cudaGetLastError();
+        return ok;
     }
+
+    bool covers(int L) const override { return L >= kC && (L + kC - 1) / kC <= max_nc_; }
 
     cudaError_t run(const void *q, const void *k, const void *v, const float *alpha, const float *beta, int L,
                     const float *S_in, float *S_out, const float *gates, int mode, float *acc, void *out,
@@ -667,7 +671,8 @@ public:
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
             !map_2d(&mut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scr.ut, kD, n * kC, kD, kC,
                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !map_2d(&mell, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scr.ell, kC, n, kC, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+            !map_2d(&mell, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scr.ell, 2 * kC, n, 2 * kC, 1,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
 
         const size_t prep_smem = sizeof(PrepSmem) + 1024, scan_smem = sizeof(ScanSmem) + 1024;
@@ -680,6 +685,14 @@ public:
             if (e != cudaSuccess) return e;
             attr_set_ = true;
         }
+        // The chunks are cut into up to kSegs segments.  The prep of segment g+1
+        // runs on an internal stream while the scan of segment g runs on `s`;
+        // the scans carry the state through a small handle-owned buffer.
+        const int segs = NC >= 4 * kSegs ? kSegs : (NC >= 8 ? 2 : 1);
+        const int per = (NC + segs - 1) / segs;
+        const size_t sstride = (size_t)BH * kD * kD;
+        cudaError_t e = cudaEventRecord(ev_[0], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(prep_stream_, ev_[0], 0);
         PrepParams pp;
         pp.alpha = alpha;
         pp.beta = beta;
@@ -688,30 +701,49 @@ public:
         pp.NC = NC;
         pp.scr = scr;
         pp.dev_err = dev_err;
-        gdn_prep_kernel<<<dim3(NC, cfg_.H, cfg_.B), 128, prep_smem, s>>>(mq, mk, mv, pp);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
         ScanParams sp;
         sp.L = L;
         sp.H = cfg_.H;
         sp.NC = NC;
-        sp.S_in = S_in;
-        sp.S_out = S_out;
         sp.gates = gates;
         sp.out_mode = mode;
         sp.acc = acc;
         sp.out = static_cast<__nv_bfloat16 *>(out);
         sp.dev_err = dev_err;
-        gdn_scan_kernel<<<dim3(cfg_.H, cfg_.B), 192, scan_smem, s>>>(mwq, mk16, mpm, mut, mell, sp);
+        int nlaunch = 0;
+        for (int g = 0; g < segs && e == cudaSuccess; ++g) {
+            const int c0 = g * per, n = min(per, NC - c0);
+            if (n <= 0) break;
+            const bool last = c0 + n >= NC;
+            pp.c_begin = c0;
+            gdn_prep_kernel<<<dim3(n, cfg_.H, cfg_.B), 128, prep_smem, prep_stream_>>>(mq, mk, mv, pp);
+            e = cudaGetLastError();
+            if (e == cudaSuccess) e = cudaEventRecord(ev_[1 + g], prep_stream_);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_[1 + g], 0);
+            sp.c_begin = c0;
+            sp.nseg = n;
+            sp.S_in = g == 0 ? S_in : s_mid_ + (g & 1) * sstride;
+            sp.S_out = last ? S_out : s_mid_ + ((g + 1) & 1) * sstride;
+            if (e == cudaSuccess)
+                gdn_scan_kernel<<<dim3(cfg_.H, cfg_.B), kScanThreads, scan_smem, s>>>(mwq, mk16, mpm, mut, mell, sp);
+            if (e == cudaSuccess) e = cudaGetLastError();
+            nlaunch += 2;
+            if (last) break;
+        }
+        if (e != cudaSuccess) return e;
         *done = true;
-        if (launches) *launches = 2;
+        if (launches) *launches = nlaunch;
         return cudaGetLastError();
     }
 
 private:
     hlta_config cfg_;
+    static constexpr int kSegs = 8;
     int max_nc_;
     void *base_ = nullptr;
+    float *s_mid_ = nullptr;
+    cudaStream_t prep_stream_ = nullptr;
+    cudaEvent_t ev_[1 + kSegs] = {};
     size_t bytes_ = 0;
     bool attr_set_ = false;
 };
