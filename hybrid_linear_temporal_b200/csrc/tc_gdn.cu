@@ -66,10 +66,11 @@ struct PrepParams {
 };
 
 struct __align__(1024) PrepSmem {
-    uint8_t kq[32768];   // 2 regions (d 0-63 / 64-127) x 128 rows: rows 0-63 K, 64-127 Q
+    // 2 regions (d 0-63 / 64-127) x 128 rows: rows 0-63 K, 64-127 Q.  Once Q has
+    // been read, its rows hold the B operands (T diag(beta g))[t][s] (region 0)
+    // and (T diag(beta))[t][s] (region 1), fp16, K-major.
+    uint8_t kq[32768];
     uint8_t v[16384];    // 2 regions x 64 rows of V
-    uint8_t b1[8192];    // (T diag(beta g))[t][s] fp16, K-major
-    uint8_t b2[8192];    // (T diag(beta))[t][s] fp16
     float A[kC][kC + 4];  // rows padded to 16 bytes
     float ell[kC], beta[kC], gam[kC], dec[kC];
     uint64_t bar_tma, bar_mma1, bar_mma2;
@@ -82,7 +83,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk16) {
     return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
 
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(128, 3)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const PrepParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -212,15 +213,19 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const uint32_t off = region * 16384 + sw128_off(row, ch);
                 uint4 *ptr = reinterpret_cast<uint4 *>(sm.kq + off);
                 const uint4 raw = *ptr;
-                const uint4 f = bf16x8_to_f16x8(raw, row < kC ? 1.f : sm.gam[row - kC]);
-                *ptr = f;
                 const int dcol = region * 64 + ch * 8;
-                if (row < kC)  // the scan's copy of K carries the decay to the chunk end
+                if (row < kC) {
+                    *ptr = bf16x8_to_f16x8(raw, 1.f);
+                    // the scan's copy of K carries the decay to the chunk end
                     *reinterpret_cast<uint4 *>(p.scr.k16 + (chunk_id * kC + row) * kD + dcol) =
                         bf16x8_to_f16x8(raw, sm.dec[row]);
-                else
-                    *reinterpret_cast<uint4 *>(p.scr.wq + (chunk_id * 128 + row) * kD + dcol) = f;
+                } else {
+                    *reinterpret_cast<uint4 *>(p.scr.wq + (chunk_id * 128 + row) * kD + dcol) =
+                        bf16x8_to_f16x8(raw, sm.gam[row - kC]);
+                }
             }
+            // Q rows are read: the solve group may now overwrite them
+            asm volatile("bar.sync 1, 128;" ::: "memory");
             for (int i = tid - kC; i < 2 * kC * 8; i += kC) {
                 const int region = i >> 9, row = (i >> 3) & 63, ch = i & 7;
                 uint4 *ptr = reinterpret_cast<uint4 *>(sm.v + region * 8192 + sw128_off(row, ch));
@@ -248,8 +253,10 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 Tc[t] = (a0 + a1) + (a2 + a3);
             }
             const float bj = sm.beta[j], bgj = sm.beta[j] * sm.gam[j];
-            __half *b1 = reinterpret_cast<__half *>(sm.b1);
-            __half *b2 = reinterpret_cast<__half *>(sm.b2);
+            // wait until the conversion group has read the Q rows
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            __half *b1 = reinterpret_cast<__half *>(sm.kq + 8192);
+            __half *b2 = reinterpret_cast<__half *>(sm.kq + 16384 + 8192);
 #pragma unroll
             for (int t = 0; t < kC; ++t) {
                 const uint32_t off = sw128_off(t, j >> 3) + (j & 7) * 2;
@@ -266,7 +273,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_after();
         const uint32_t idesc = idesc_f16_f32(128, 64, 1, 0);
         const uint32_t kb = smem_u32(sm.kq), vb = smem_u32(sm.v);
-        const uint32_t b1 = smem_u32(sm.b1), b2 = smem_u32(sm.b2);
+        const uint32_t b1 = smem_u32(sm.kq + 8192), b2 = smem_u32(sm.kq + 16384 + 8192);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             umma_ss(tmem + 64, smem_desc_sw128(kb + kk * 2048, 16384, 1024), smem_desc_sw128(b1 + kk * 32, 16, 1024),
@@ -763,3 +770,4 @@ TcGdn *TcGdn::create(const hlta_config &cfg, long long max_seq_len) {
 }
 
 }  // namespace hlta
+
