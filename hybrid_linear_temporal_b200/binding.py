@@ -69,6 +69,7 @@ def load_library(path: str | None = None):
         "hlta_device_status": ([vp], st),
         "hlta_profile_enable": ([vp, i], st),
         "hlta_profile_read": ([vp, ctypes.POINTER(ProfileData)], st),
+        "hlta_gdn_forward_noalloc": ([i, i, i, vp, vp, vp, fp, fp, fp, fp, fp, vp, vp], st),
         "hlta_last_error": ([], ctypes.c_char_p),
         "hlta_version": ([], i),
     }
@@ -101,6 +102,22 @@ def _stream(stream):
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def gdn_forward_noalloc(q, k, v, alpha, beta, gates, S0=None, S_out=None, out=None, stream=None):
+    """Memory branch without device allocation (hlta_gdn_forward_noalloc).
+
+    For callers that must not allocate device memory while running; the scratch
+    is a static array in the library.  Tensors as for HLTA.forward with
+    d_k = d_v = 128, bf16; returns out = g[h,2] * o_t."""
+    import torch
+    lib = load_library()
+    B, L, H, _ = q.shape
+    if out is None:
+        out = torch.empty_like(v)
+    _check(lib, lib.hlta_gdn_forward_noalloc(B, L, H, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                             _ptr(gates), _ptr(S0), _ptr(S_out), _ptr(out), _stream(stream)))
+    return out
 
 
 class HLTA:

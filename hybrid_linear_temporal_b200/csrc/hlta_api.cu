@@ -63,6 +63,11 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+namespace hlta {
+// Sets the thread-local message returned by hlta_last_error() (empty clears it).
+void set_last_error(const char *msg) { g_last_error = msg ? msg : ""; }
+}  // namespace hlta
+
 struct hlta_handle {
     hlta_config cfg;
     int device = 0;

@@ -62,6 +62,9 @@ struct RingAppendArgs {
     int n, B, H, d_k, d_v, elem_bytes;
 };
 
+// Sets the thread-local message returned by hlta_last_error() (empty clears it).
+void set_last_error(const char *msg);
+
 cudaError_t launch_attn_simt(const AttnSimtArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_gdn_recurrent(const GdnRecArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_ring_append(const RingAppendArgs &a, cudaStream_t s);

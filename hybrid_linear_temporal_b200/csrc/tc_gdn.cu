@@ -771,3 +771,146 @@ TcGdn *TcGdn::create(const hlta_config &cfg, long long max_seq_len) {
 
 }  // namespace hlta
 
+// =====================================================================
+// hlta_gdn_forward_noalloc: the chunked memory branch without any device
+// allocation.  Some callers may not allocate device memory once they are
+// running -- for example a control loop under a fixed memory budget that
+// reserves everything at start-up, or code inside a foreign allocator that
+// forbids cudaMalloc.  They cannot create a handle (hlta_create allocates), so
+// this entry point takes every size as an argument and runs the same prep and
+// scan kernels on a scratch that lives in a file-scope __device__ array.
+//
+// The array is part of the library image: every GPU that loads the library
+// holds its 96 MiB until the process exits.  All calls share it and it keeps
+// the previous call's contents; each call clears what must start at zero (the
+// device error word).  Calls whose executions overlap on the GPU (for example
+// on two streams) race on it and must be ordered by the caller.
+// =====================================================================
+#include <mutex>
+
+#include "hlta.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 96ull << 20;
+// 256-byte aligned; the error word sits in the first 256 bytes, the chunk
+// scratch starts at byte 256 (TMA needs 16-byte aligned bases, kept here).
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_base[kNoAllocMaxDevices];  // device address of the array, per device
+
+constexpr size_t kNoAllocChunkBytes = hlta::kWQBytes + hlta::kK16Bytes + hlta::kPmBytes + hlta::kUtBytes +
+                                      hlta::kEllBytes;
+
+hlta_status noalloc_fail(hlta_status st, const char *msg) {
+    hlta::set_last_error(msg);
+    return st;
+}
+
+}  // namespace
+
+extern "C" HLTA_API hlta_status hlta_gdn_forward_noalloc(int B, int L, int H, const void *q, const void *k,
+                                                         const void *v, const float *alpha, const float *beta,
+                                                         const float *gates, const float *S0, float *S_out,
+                                                         void *out, void *stream) {
+    using namespace hlta;
+    if (B < 1 || H < 1 || L < kC)
+        return noalloc_fail(HLTA_ERR_INVALID_ARG, "hlta_gdn_forward_noalloc: need B >= 1, H >= 1, L >= 64");
+    const void *ptrs[] = {q, k, v, alpha, beta, gates, out};
+    for (const void *ptr : ptrs)
+        if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 15u))
+            return noalloc_fail(HLTA_ERR_INVALID_ARG,
+                                "hlta_gdn_forward_noalloc: a required pointer is NULL or not 16-byte aligned");
+    if ((S0 && (reinterpret_cast<uintptr_t>(S0) & 15u)) || (S_out && (reinterpret_cast<uintptr_t>(S_out) & 15u)))
+        return noalloc_fail(HLTA_ERR_INVALID_ARG, "hlta_gdn_forward_noalloc: S0/S_out not 16-byte aligned");
+    const int NC = (L + kC - 1) / kC;
+    const size_t n = (size_t)B * H * NC;
+    if (256 + n * kNoAllocChunkBytes > kNoAllocScratchBytes)
+        return noalloc_fail(HLTA_ERR_UNSUPPORTED,
+                            "hlta_gdn_forward_noalloc: B*H*ceil(L/64) exceeds the 1110 chunk-heads of the "
+                            "static 96 MiB scratch");
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+        return noalloc_fail(HLTA_ERR_CUDA, "hlta_gdn_forward_noalloc: no usable current device");
+    char *base = nullptr;
+    {
+        // once per device, with that device current: the device address of the
+        // array (the host-side symbol is not a device address) and the kernels'
+        // shared-memory limits
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_base[dev]) {
+            void *ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+                cudaGetLastError();
+                return noalloc_fail(HLTA_ERR_CUDA, "hlta_gdn_forward_noalloc: cudaGetSymbolAddress failed");
+            }
+            if (cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(sizeof(PrepSmem) + 1024)) != cudaSuccess ||
+                cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(sizeof(ScanSmem) + 1024)) != cudaSuccess) {
+                cudaGetLastError();
+                return noalloc_fail(HLTA_ERR_CUDA, "hlta_gdn_forward_noalloc: cudaFuncSetAttribute failed");
+            }
+            g_noalloc_base[dev] = ptr;
+        }
+        base = static_cast<char *>(g_noalloc_base[dev]);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int *dev_err = reinterpret_cast<int *>(base);
+    GdnScratch scr;
+    char *p = base + 256;
+    scr.wq = reinterpret_cast<__half *>(p);
+    p += n * kWQBytes;
+    scr.k16 = reinterpret_cast<__half *>(p);
+    p += n * kK16Bytes;
+    scr.pm = reinterpret_cast<__half *>(p);
+    p += n * kPmBytes;
+    scr.ut = reinterpret_cast<float *>(p);
+    p += n * kUtBytes;
+    scr.ell = reinterpret_cast<float *>(p);
+
+    CUtensorMap mq, mk, mv, mwq, mk16, mpm, mut, mell;
+    if (!map_tokens(&mq, q, H, L, B) || !map_tokens(&mk, k, H, L, B) || !map_tokens(&mv, v, H, L, B) ||
+        !map_2d(&mwq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scr.wq, kD, n * 128, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mk16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scr.k16, kD, n * kC, 64, kC, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mpm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scr.pm, kC, n * kC, 64, kC, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scr.ut, kD, n * kC, kD, kC, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !map_2d(&mell, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scr.ell, 2 * kC, n, 2 * kC, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return noalloc_fail(HLTA_ERR_CUDA, "hlta_gdn_forward_noalloc: tensor map encoding failed");
+
+    if (cudaMemsetAsync(dev_err, 0, sizeof(int), s) != cudaSuccess) {
+        cudaGetLastError();
+        return noalloc_fail(HLTA_ERR_CUDA, "hlta_gdn_forward_noalloc: clearing the error word failed");
+    }
+    PrepParams pp;
+    pp.alpha = alpha;
+    pp.beta = beta;
+    pp.L = L;
+    pp.H = H;
+    pp.NC = NC;
+    pp.c_begin = 0;
+    pp.scr = scr;
+    pp.dev_err = dev_err;
+    gdn_prep_kernel<<<dim3(NC, H, B), 128, sizeof(PrepSmem) + 1024, s>>>(mq, mk, mv, pp);
+    ScanParams sp;
+    sp.L = L;
+    sp.H = H;
+    sp.NC = NC;
+    sp.c_begin = 0;
+    sp.nseg = NC;
+    sp.S_in = S0;
+    sp.S_out = S_out;
+    sp.gates = gates;
+    sp.out_mode = OUT_FINAL_ONLY;
+    sp.acc = nullptr;
+    sp.out = static_cast<__nv_bfloat16 *>(out);
+    sp.dev_err = dev_err;
+    gdn_scan_kernel<<<dim3(H, B), kScanThreads, sizeof(ScanSmem) + 1024, s>>>(mwq, mk16, mpm, mut, mell, sp);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return noalloc_fail(HLTA_ERR_CUDA, cudaGetErrorString(e));
+    hlta::set_last_error("");
+    return HLTA_OK;
+}

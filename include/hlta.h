@@ -188,6 +188,29 @@ HLTA_API hlta_status hlta_profile_enable(hlta_handle *h, int enable);
 /* Synchronise the handle's device and report the records since enabling. */
 HLTA_API hlta_status hlta_profile_read(hlta_handle *h, hlta_profile_data *out);
 
+/*
+ * hlta_gdn_forward_noalloc: the memory branch alone (the chunked gated delta
+ * memory of hlta_forward with branches = HLTA_BRANCH_GDN) for callers that must
+ * not allocate device memory once running -- a control loop with a fixed memory
+ * budget reserved at start-up, or code under an allocator that forbids
+ * cudaMalloc -- and therefore cannot create a handle.  It has no counterpart on
+ * the pages; it exists only so that such callers can run the layer's memory.
+ *   Sizes come as arguments; head dims are fixed at d_k = d_v = 128, dtype bf16,
+ *   chunk 64.  q, k, v: [B,L,H,128] bf16; alpha, beta: [B,L,H] f32; gates: [H,3]
+ *   f32 (only g[h,2] is used); S0, S_out: [B,H,128,128] f32 or NULL; out:
+ *   [B,L,H,128] bf16 receives g[h,2] * o_t.  Device pointers, 16-byte aligned,
+ *   owned by the caller.  Requires L >= 64 and B*H*ceil(L/64) <= 1110.
+ * It allocates nothing: its scratch is a 96 MiB array in the library image,
+ * which every GPU that loads the library holds until the process exits.  The
+ * first call on a device looks up that array's device address and sets kernel
+ * attributes; make that first call before any stream capture.  All calls share
+ * the array: calls that overlap on the GPU race and must be ordered by the
+ * caller.  Enqueued on `stream`; INVALID_ARG / UNSUPPORTED (too large) / CUDA.
+ */
+HLTA_API hlta_status hlta_gdn_forward_noalloc(int B, int L, int H, const void *q, const void *k, const void *v,
+                                              const float *alpha, const float *beta, const float *gates,
+                                              const float *S0, float *S_out, void *out, void *stream);
+
 /* Thread-local message describing the last failed call ("" if none). */
 HLTA_API const char *hlta_last_error(void);
 
