@@ -223,10 +223,10 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
     geo[1].dil = c.dswa_dilation;
     geo[1].w = c.dswa_window;
     const bool want_attn[2] = {(branches & 1u) != 0, (branches & 2u) != 0};
-    // Concurrent schedule: the memory branch (two kernels, one of them a
-    // sequential scan on B*H SMs) runs on the side stream into its own
-    // accumulator while SWA runs on `s`; the last attention branch waits for it
-    // and adds both accumulators in its epilogue.
+    // Concurrent schedule: the memory branch (prep kernels and a sequential
+    // scan on B*H SMs) runs on the side stream into its own accumulator while
+    // SWA and DSWA run on `s` into theirs; after the join one elementwise pass
+    // writes out = acc + acc2 (the gated sum of all three branches).
     const bool overlap = one_shot && (branches & 4u) && (want_attn[0] || want_attn[1]) && h->side &&
                          h->acc2 && h->tc_gdn && h->tc_gdn->covers(nq) && h->tc_attn &&
                          (!want_attn[0] || h->tc_attn->covers(nq, geo[0])) &&
@@ -246,22 +246,23 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
             ps.done(launches);
         }
         CK(cudaEventRecord(h->ev_join, h->side));
-        const int na = (int)want_attn[0] + (int)want_attn[1];
+        // both attention branches run on `s` while the memory branch runs
         int idx = 0;
         for (int br = 0; br < 2; ++br) {
             if (!want_attn[br]) continue;
-            const bool last = idx == na - 1;
-            if (last) CK(cudaStreamWaitEvent(s, h->ev_join, 0));
-            const int mode = na == 1 ? hlta::OUT_FINAL_ONLY : (last ? hlta::OUT_FINAL : hlta::OUT_STORE);
             ProfScope ps(h, br, s);
             bool done = false;
-            cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, geo[br], in.gates, br, mode, h->acc,
-                                            last ? h->acc2 : nullptr, out, h->dev_err, s, &done);
+            cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, geo[br], in.gates, br,
+                                            idx == 0 ? hlta::OUT_STORE : hlta::OUT_ADD, h->acc, nullptr, out,
+                                            h->dev_err, s, &done);
             if (e != cudaSuccess || !done)
                 return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
             ps.done(1);
             ++idx;
         }
+        CK(cudaStreamWaitEvent(s, h->ev_join, 0));
+        CK(hlta::launch_sum_to_bf16(h->acc, h->acc2, out, (size_t)c.B * nq * c.H * c.d_v, s));
+        if (h->prof) h->prof_launches += 1;
         return HLTA_OK;
     }
     for (int idx = 0; idx < n; ++idx) {
@@ -397,7 +398,11 @@ hlta_status hlta_create(const hlta_config *cfg, hlta_handle **out) {
         h->tc_gdn = hlta::TcGdn::create(*cfg, cfg->max_seq_len);
         if (h->tc_attn && h->tc_gdn) {
             const size_t acc2_bytes = (size_t)cfg->B * cfg->max_seq_len * cfg->H * cfg->d_v * sizeof(float);
-            if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
+            // the memory branch is latency-bound and on the critical path: its stream
+            // gets the highest priority so its CTAs are scheduled first as SMs free up
+            int prio_lo = 0, prio_hi = 0;
+            cudaDeviceGetStreamPriorityRange(&prio_lo, &prio_hi);
+            if (cudaStreamCreateWithPriority(&h->side, cudaStreamNonBlocking, prio_hi) != cudaSuccess ||
                 cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
                 cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess ||
                 cudaMalloc((void **)&h->acc2, acc2_bytes) != cudaSuccess) {

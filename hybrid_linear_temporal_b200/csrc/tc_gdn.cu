@@ -637,8 +637,10 @@ public:
         const size_t n = (size_t)cfg_.B * cfg_.H * max_nc_;
         bytes_ = n * (kWQBytes + kK16Bytes + kPmBytes + kUtBytes + kEllBytes);
         const size_t sbytes = (size_t)cfg_.B * cfg_.H * kD * kD * sizeof(float);
+        int prio_lo = 0, prio_hi = 0;
+        cudaDeviceGetStreamPriorityRange(&prio_lo, &prio_hi);
         bool ok = cudaMalloc(&base_, bytes_) == cudaSuccess && cudaMalloc(&s_mid_, 2 * sbytes) == cudaSuccess &&
-                  cudaStreamCreateWithFlags(&prep_stream_, cudaStreamNonBlocking) == cudaSuccess;
+                  cudaStreamCreateWithPriority(&prep_stream_, cudaStreamNonBlocking, prio_hi) == cudaSuccess;
         for (auto &e : ev_) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
         if (!ok) cudaGetLastError();
         return ok;
