@@ -15,18 +15,24 @@
 //
 // One CTA (one per SM) handles two adjacent 128-row query tiles of a segment,
 // which share every K/V tile:
-//   warp 0      TMA producer: Q0, Q1, then K_t and V_t through a 4-slot ring
+//   warp 0      TMA producer: Q0, Q1, then K_t and V_t through a 5-slot ring
 //   warp 1      TMEM allocation (512 columns); lane 0 issues tcgen05.mma
 //                 S_j = Q_j K_t^T   (SS form, 128x128x128, fp32 in TMEM)
 //                 O_j += P_j V_t    (TS form: P_j read from TMEM, V_t MN-major)
-//               in the order QK0, QK1, PV0, PV1, so one tile's softmax overlaps
-//               the other tile's MMAs
+//               in the order PV0(t), QK0(t+1), PV1(t), QK1(t+1), so that the
+//               softmax of one query tile runs under the other tile's MMAs
 //   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: thread = query
-//               row = TMEM lane.  Online softmax in the log2 domain with a
-//               lazily moved reference maximum (O_j is rescaled in TMEM only when
-//               a row maximum grows by more than 2^8); P_j is written back over
-//               S_j as bf16; the epilogue scales O_j by gate/l and writes rows.
-// TMEM: S0 cols 0-127, S1 128-255, O0 256-383, O1 384-511.
+//               row = TMEM lane.  Each row of S_j is read from TMEM once; online
+//               softmax in the log2 domain with a lazily moved reference maximum
+//               (O_j is rescaled in TMEM only when a row maximum grows by more
+//               than 2^8); P_j is written back as bf16 over the first 64 columns
+//               of S_j; the epilogue scales O_j by gate/l and writes rows.
+// TMEM: S0/P0 cols 0-127, S1/P1 128-255, O0 256-383, O1 384-511.
+// P_j aliases S_j: QK_j(t+1) is issued after PV_j(t) by the same thread, and
+// the tensor pipe executes one thread's MMAs in issue order, so PV_j(t) has read
+// P_j before QK_j(t+1) overwrites it.  For the same reason the commit that
+// signals S_j(t) also covers PV_j(t-1): the softmax may rescale O_j as soon as
+// S_j(t) is ready.
 // Key tiles never straddle a segment; a tile is skipped for a query tile whose
 // band it misses, and tiles crossing a band edge or a segment end are masked
 // per element.
@@ -49,7 +55,7 @@ constexpr int kBN = 128;   // keys per tile
 constexpr int kD = 128;    // head dim (d_k = d_v)
 constexpr int kMaxKT = 40;
 constexpr int kThreads = 320;
-constexpr int kSlots = 3;                        // K/V ring slots (one 128x128 bf16 tile each)
+constexpr int kSlots = 5;                        // K/V ring slots (one 128x128 bf16 tile each)
 constexpr uint32_t kTileBytes = kBN * kD * 2;    // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-column TMA box
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
@@ -79,8 +85,7 @@ struct TcAttnParams {
 struct __align__(16) Smem {
     uint8_t q[kQT][kTileBytes];
     uint8_t kv[kSlots][kTileBytes];
-    uint8_t pm[kQT][kTileBytes];  // P_j, bf16, K-major 128B-swizzled (A operand of P V)
-    uint64_t bar_q, full[kSlots], empty[kSlots], bar_s[kQT], bar_p[kQT], bar_pv[kQT];
+    uint64_t bar_q, full[kSlots], empty[kSlots], bar_s[kQT], bar_p[kQT], bar_o;
     uint32_t tmem_base;
     int abort;
     int nkt;
@@ -144,76 +149,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
-// Row maximum of the raw scores in TMEM columns [col, col+128) of this thread's
-// lane.  The softmax scale is positive, so the maximum is taken before scaling.
-// kMask: only columns in [lo, hi] count (band edges, segment ends).
-template <bool kMask>
-__device__ __forceinline__ float tile_row_max(uint32_t taddr, int lo, int hi) {
-    float m[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
-#pragma unroll
-    for (int hlf = 0; hlf < 2; ++hlf) {
-        uint32_t r[2][32];
-        tmem_ld32(taddr + hlf * 64, r[0]);
-        tmem_ld32(taddr + hlf * 64 + 32, r[1]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                float x0 = __uint_as_float(r[c][j]), x1 = __uint_as_float(r[c][j + 1]);
-                if (kMask) {
-                    const int col = hlf * 64 + c * 32 + j;
-                    if (col < lo || col > hi) x0 = -INFINITY;
-                    if (col + 1 < lo || col + 1 > hi) x1 = -INFINITY;
-                }
-                const int a = (j >> 1) & 7;
-                m[a] = max3f(m[a], x0, x1);
-            }
-    }
-    return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
-}
-
-// p = 2^(s*scale - m) over TMEM columns [col, col+128), written as bf16 row
-// `row` of a K-major 128B-swizzled P tile in shared memory (keys 0-63 in the
-// first 16 KB region, keys 64-127 in the second).  Returns the row sum of p.
-template <bool kMask>
-__device__ __forceinline__ float tile_exp_store(uint32_t taddr, float scale, float m, int lo, int hi,
-                                                uint8_t *ptile, int row) {
-    float sum[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sum[i] = 0.f;
-#pragma unroll
-    for (int hlf = 0; hlf < 2; ++hlf) {
-        uint32_t a[32], b[32], pk[32];
-        tmem_ld32(taddr + hlf * 64, a);
-        tmem_ld32(taddr + hlf * 64 + 32, b);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 64; j += 2) {
-            const uint32_t u0 = j < 32 ? a[j] : b[j - 32];
-            const uint32_t u1 = j < 32 ? a[j + 1] : b[j - 31];
-            float x0 = fmaf(__uint_as_float(u0), scale, -m);
-            float x1 = fmaf(__uint_as_float(u1), scale, -m);
-            if (kMask) {
-                const int col = hlf * 64 + j;
-                if (col < lo || col > hi) x0 = -INFINITY;
-                if (col + 1 < lo || col + 1 > hi) x1 = -INFINITY;
-            }
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            sum[(j >> 1) & 7] += p0 + p1;
-            pk[j >> 1] = pack_bf16x2(p0, p1);
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint32_t off = hlf * kHalfBytes + row * 128 + ((c ^ (row & 7)) << 4);
-            *reinterpret_cast<uint4 *>(ptile + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-    }
-    return ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const TcAttnParams p) {
@@ -263,8 +198,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int j = 0; j < kQT; ++j) {
             mbar_init(&sm.bar_s[j], 1);
             mbar_init(&sm.bar_p[j], 128);
-            mbar_init(&sm.bar_pv[j], 1);
         }
+        mbar_init(&sm.bar_o, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -311,35 +246,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        // Order per key tile t: PV0(t), QK0(t+1), PV1(t), QK1(t+1), so that the
-        // softmax of one query tile runs under the other tile's MMAs.  P_j lives
-        // in shared memory, so S_j may be rewritten as soon as PV_j(t) is issued.
-        if (lane == 0 && !*abort) {
+        // Per key tile t: PV0(t), QK0(t+1), PV1(t), QK1(t+1).  QK_j(t+1) reuses
+        // S_j's columns, which hold P_j(t): it is issued after PV_j(t).
+        if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
             int npv[kQT] = {0, 0};
-            bool live = mbar_wait(&sm.bar_q, 0, abort, p.dev_err);
-            // QK_j for key tile t (K_t must be resident)
-            auto issue_qk = [&](int t) {
-                const uint32_t ka = smem_u32(sm.kv[(2 * t) % kSlots]);
+            bool live = !*abort && mbar_wait(&sm.bar_q, 0, abort, p.dev_err);
+            // S_j = Q_j K^T for the key tile in ring slot `ks`
+            auto issue_qk = [&](int j, uint32_t ka) {
+                tc_fence_after();
+                const uint32_t qa = smem_u32(sm.q[j]);
 #pragma unroll
-                for (int j = 0; j < kQT; ++j) {
-                    if (!sm.kt[t].use[j]) continue;
-                    tc_fence_after();
-                    const uint32_t qa = smem_u32(sm.q[j]);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
-                        umma_ss(tmem + j * 128, smem_desc_sw128(qa + off, 16, 1024),
-                                smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&sm.bar_s[j]);
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
+                    umma_ss(tmem + j * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
+                            idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&sm.empty[(2 * t) % kSlots]);
+                umma_commit(&sm.bar_s[j]);
             };
             if (live && nkt > 0) {
                 live = mbar_wait(&sm.full[0], 0, abort, p.dev_err);
-                if (live) issue_qk(0);
+                if (live) {
+                    const uint32_t ka = smem_u32(sm.kv[0]);
+#pragma unroll
+                    for (int j = 0; j < kQT; ++j)
+                        if (sm.kt[0].use[j]) issue_qk(j, ka);
+                    umma_commit(&sm.empty[0]);
+                }
             }
             for (int t = 0; t < nkt && live; ++t) {
                 const KeyTile kt = sm.kt[t];
@@ -347,52 +281,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (!(live = mbar_wait(&sm.full[sv], (uv / kSlots) & 1, abort, p.dev_err))) break;
                 const uint32_t va = smem_u32(sm.kv[sv]);
                 const bool more = t + 1 < nkt;
+                const int uk = 2 * (t + 1), sk = uk % kSlots;
                 bool k_ready = false;
-                uint32_t ka = 0u;
 #pragma unroll
                 for (int j = 0; j < kQT; ++j) {
                     if (kt.use[j]) {
                         if (!(live = mbar_wait(&sm.bar_p[j], npv[j] & 1, abort, p.dev_err))) break;
                         tc_fence_after();
-                        const uint32_t pa = smem_u32(sm.pm[j]);
 #pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk) {
-                            const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
-                            umma_ss(tmem + 256 + j * 128, smem_desc_sw128(pa + off, 16, 1024),
+                        for (int kk = 0; kk < kBN / 16; ++kk)
+                            umma_ts(tmem + 256 + j * 128, tmem + j * 128 + kk * 8,
                                     smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
                                     (npv[j] > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(&sm.bar_pv[j]);
                         ++npv[j];
                     }
                     if (more && sm.kt[t + 1].use[j]) {
                         if (!k_ready) {
-                            const int uk = 2 * (t + 1);
-                            if (!(live = mbar_wait(&sm.full[uk % kSlots], (uk / kSlots) & 1, abort, p.dev_err)))
-                                break;
-                            ka = smem_u32(sm.kv[uk % kSlots]);
+                            if (!(live = mbar_wait(&sm.full[sk], (uk / kSlots) & 1, abort, p.dev_err))) break;
                             k_ready = true;
                         }
-                        tc_fence_after();
-                        const uint32_t qa = smem_u32(sm.q[j]);
-#pragma unroll
-                        for (int kk = 0; kk < kD / 16; ++kk) {
-                            const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
-                            umma_ss(tmem + j * 128, smem_desc_sw128(qa + off, 16, 1024),
-                                    smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&sm.bar_s[j]);
+                        issue_qk(j, smem_u32(sm.kv[sk]));
                     }
                 }
                 if (!live) break;
                 umma_commit(&sm.empty[sv]);
-                if (k_ready) umma_commit(&sm.empty[(2 * (t + 1)) % kSlots]);
+                if (more) {
+                    // a K tile no query tile uses still has to be released
+                    if (!k_ready && !(live = mbar_wait(&sm.full[sk], (uk / kSlots) & 1, abort, p.dev_err))) break;
+                    umma_commit(&sm.empty[sk]);
+                }
             }
+            // every MMA of this CTA is complete once bar_o fires
+            umma_commit(&sm.bar_o);
             if (*abort) {
                 int dummy = 0;
                 volatile int *no_abort = &dummy;
-                for (int j = 0; j < kQT; ++j)
-                    if (npv[j] > 0) mbar_wait(&sm.bar_pv[j], (npv[j] - 1) & 1, no_abort, nullptr);
+                mbar_wait(&sm.bar_o, 0, no_abort, nullptr);
             }
         }
     } else {
@@ -403,9 +327,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t colS = j * 128, colO = 256 + j * 128;
         const int nqj = j == 0 ? nq0 : nq1;
-        const int lo_q = r_min + j * kBM;
-        const int hi_q = lo_q + nqj - 1;
-        const int r_q = lo_q + row;
+        const int r_q = r_min + j * kBM + row;
+        const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l_run = 0.f;
         int n = 0;
         bool ok = !*abort;
@@ -420,56 +343,77 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            int lo = 0, hi = kBN - 1;
+            uint32_t s[128];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                tmem_ld32(tl + colS + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * i]));
+            tmem_wait_ld();
             if (!full) {
-                lo = max(0, r_q - p.w + 1 - rbase);
-                hi = min(kvalid - 1, r_q - rbase);
+                const int lo = max(0, r_q - p.w + 1 - rbase);
+                const int hi = min(kvalid - 1, r_q - rbase);
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
             }
-            const float mraw = full ? tile_row_max<false>(tl + colS, lo, hi) : tile_row_max<true>(tl + colS, lo, hi);
-            const float mx = mraw * p.scale_log2;  // -inf stays -inf
-            float scale = 1.f;
+            // the softmax scale is positive: take the maximum of the raw scores
+            float mx;
+            {
+                float mm8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mm8[i] = __uint_as_float(s[i]);
+#pragma unroll
+                for (int c = 8; c < 128; c += 16)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        mm8[i] = max3f(mm8[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
+                mx = max3f(max3f(mm8[0], mm8[1], mm8[2]), max3f(mm8[3], mm8[4], mm8[5]), fmaxf(mm8[6], mm8[7]));
+                mx *= sl2;  // -inf stays -inf
+            }
+            float alpha = 1.f;
             bool moved = false;
             if (mx > m_ref + kRescaleThreshold) {
-                scale = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+                alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
                 m_ref = mx;
                 moved = true;
             }
-            l_run *= scale;
-            // O_j holds earlier tiles' contributions once n > 0: rescale it
-            if (n > 0 && __any_sync(0xffffffffu, moved)) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_pv[j], (n - 1) & 1, abort, p.dev_err))) {
-                    ok = false;
-                    break;
+            const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+            // P = 2^(s*scale - m) as bf16 over columns 0-63 of S_j
+            float sum[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum[i] = 0.f;
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const float p0 = ex2(fmaf(__uint_as_float(s[hlf * 64 + c]), sl2, neg_m));
+                    const float p1 = ex2(fmaf(__uint_as_float(s[hlf * 64 + c + 1]), sl2, neg_m));
+                    sum[(c >> 1) & 7] += p0 + p1;
+                    pk[c >> 1] = pack_bf16x2(p0, p1);
                 }
-                tc_fence_after();
+                tmem_st32(tl + colS + hlf * 32, pk);
+            }
+            // O_j holds earlier tiles' contributions once n > 0; PV_j(t-1) is complete
+            // (it was issued before QK_j(t), whose commit fired)
+            if (n > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
                     tmem_ld32(tl + colO + c * 32, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) o[jj] = __float_as_uint(__uint_as_float(o[jj]) * scale);
+                    for (int jj = 0; jj < 32; ++jj) o[jj] = __float_as_uint(__uint_as_float(o[jj]) * alpha);
                     tmem_st32(tl + colO + c * 32, o);
                 }
-                tmem_wait_st();
             }
-            const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            // P_j's buffer is read by PV_j of the previous tile: wait for it (in the
-            // steady state it completed long ago)
-            if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_pv[j], (n - 1) & 1, abort, p.dev_err))) {
-                ok = false;
-                break;
-            }
-            const float lsum = full ? tile_exp_store<false>(tl + colS, p.scale_log2, m_use, lo, hi, sm.pm[j], row)
-                                    : tile_exp_store<true>(tl + colS, p.scale_log2, m_use, lo, hi, sm.pm[j], row);
-            l_run += lsum;
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.bar_p[j]);
+            l_run = fmaf(l_run, alpha,
+                         ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
             ++n;
         }
-        (void)hi_q;
-        if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.bar_pv[j], (n - 1) & 1, abort, p.dev_err))) {
+        if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.bar_o, 0, abort, p.dev_err))) {
             tc_fence_after();
             const int tok = seg_f * p.Pseg + s0 + j * kBM + row;
             const size_t base = (((size_t)b * p.L + tok) * p.H + h) * kD;
