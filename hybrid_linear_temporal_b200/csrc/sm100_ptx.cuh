@@ -59,27 +59,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not yet complete is suspended
+// (it takes no issue slots) until the phase completes or about `ns`
+// nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr uint32_t kSuspendNs = 100000;  // 0.1 ms per suspended try
+
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises *abort / the device error word) if it did not within kWaitNs, or if
 // another thread of the CTA -- or any CTA of any launch, through the device
 // error word -- already gave up, so one failure ends the whole grid quickly.
+// Waiting threads are suspended in the barrier instead of spinning, so that
+// they leave the issue slots to the warps that share their scheduler.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int *dev_err) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (*abort) return false;
-            if (dev_err && *reinterpret_cast<volatile int *>(dev_err) != 0) {
-                *abort = 1;
-                return false;
-            }
-            if (globaltimer() - t0 > kWaitNs) {
-                *abort = 1;
-                if (dev_err) atomicExch(dev_err, DEVERR_TIMEOUT);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
+        if (*abort) return false;
+        if (dev_err && *reinterpret_cast<volatile int *>(dev_err) != 0) {
+            *abort = 1;
+            return false;
+        }
+        if (globaltimer() - t0 > kWaitNs) {
+            *abort = 1;
+            if (dev_err) atomicExch(dev_err, DEVERR_TIMEOUT);
+            return false;
         }
     }
 }

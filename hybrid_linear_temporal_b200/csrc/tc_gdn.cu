@@ -11,17 +11,19 @@
 //   S_C = g_C S0 + U^T diag(e^{l_C-l}) K.
 // Two kernels:
 //   gdn_prep_kernel  (one CTA per chunk, all chunks in parallel): [K;Q] K^T on
-//       tcgen05 (bf16), the decay masks, T by forward substitution on CUDA cores,
-//       then W^T = K^T (T diag(beta g))^T and U~^T = V^T (T diag(beta))^T as fp16
+//       tcgen05 (bf16), the decay masks, T by blocked forward substitution on
+//       CUDA cores (16x16 diagonal blocks, then the block diagonals below), then
+//       W^T = K^T (T diag(beta g))^T and U~^T = V^T (T diag(beta))^T as fp16
 //       tcgen05 MMAs.  Writes W and g*Q (fp16), K (fp16), Pm (fp16), U~ (fp32)
 //       and l to a per-chunk scratch.
 //   gdn_scan_kernel  (one CTA per (b, h), chunks in sequence): the d_v = 128 rows
-//       of the state are the MMA's M dimension.  Per chunk:
-//         [S0 W^T | S0 (gQ)^T]  = S16 x [W; gQ]^T      (S16: fp16 copy of S in TMEM)
-//         U^T = U~^T - S0 W^T                         (CUDA cores, fp32)
-//         O^T += U^T Pm^T,  D = U^T (diag(e^{l_C-l}) K)   (A operand read from TMEM)
-//         S = g_C S + D  (fp32, held in the math warps' registers), S16 = fp16(S),
-//         outputs written per token.
+//       of the state are the MMA's M dimension.  Per chunk the serial chain is
+//         S0 W^T = S16 W^T                 (S16: fp16 copy of S in TMEM)
+//         U^T = U~^T - S0 W^T               (CUDA cores, fp32)
+//         D = U^T (diag(e^{l_C-l}) K)        (A operand read from TMEM)
+//         S = g_C S + D  (fp32, held in the math warps' registers), S16 = fp16(S)
+//       and the output half runs beside it: O^T = S16 (gQ)^T + U^T Pm^T, written
+//       per token.
 // Internal operands are fp16 (11-bit mantissa) with fp32 accumulation; every
 // value they carry is bounded (unit keys, alpha in (0,1], beta in [0,1]).
 #include <cuda_bf16.h>
@@ -71,7 +73,8 @@ struct __align__(1024) PrepSmem {
     // and (T diag(beta))[t][s] (region 1), fp16, K-major.
     uint8_t kq[32768];
     uint8_t v[16384];    // 2 regions x 64 rows of V
-    float A[kC][kC + 4];  // rows padded to 16 bytes
+    float A[kC][kC + 4];  // rows padded to 16 bytes; T^T is built in the upper triangle
+    float Y[3 * 256];     // block products of the triangular inverse
     float ell[kC], beta[kC], gam[kC], dec[kC];
     uint64_t bar_tma, bar_mma1, bar_mma2;
     uint32_t tmem_base;
@@ -205,63 +208,104 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
 
     if (!*abort) {
-        if (tid >= kC) {
-            // threads 64..127, while 0..63 solve: bf16 -> fp16 in place (Q rows scaled
-            // by g_t), and the K and g*Q copies to the scratch
-            for (int i = tid - kC; i < 2 * 128 * 8; i += kC) {
-                const int region = i >> 10, row = (i >> 3) & 127, ch = i & 7;
-                const uint32_t off = region * 16384 + sw128_off(row, ch);
-                uint4 *ptr = reinterpret_cast<uint4 *>(sm.kq + off);
-                const uint4 raw = *ptr;
-                const int dcol = region * 64 + ch * 8;
-                if (row < kC) {
-                    *ptr = bf16x8_to_f16x8(raw, 1.f);
-                    // the scan's copy of K carries the decay to the chunk end
-                    *reinterpret_cast<uint4 *>(p.scr.k16 + (chunk_id * kC + row) * kD + dcol) =
-                        bf16x8_to_f16x8(raw, sm.dec[row]);
-                } else {
-                    *reinterpret_cast<uint4 *>(p.scr.wq + (chunk_id * 128 + row) * kD + dcol) =
-                        bf16x8_to_f16x8(raw, sm.gam[row - kC]);
+        // bf16 -> fp16 in place (the fp16 MMA below takes K and V), the scan's
+        // copies of K (carrying the decay to the chunk end) and of g*Q
+        for (int i = tid; i < 2 * 128 * 8; i += 128) {
+            const int region = i >> 10, row = (i >> 3) & 127, ch = i & 7;
+            const uint32_t off = region * 16384 + sw128_off(row, ch);
+            uint4 *ptr = reinterpret_cast<uint4 *>(sm.kq + off);
+            const uint4 raw = *ptr;
+            const int dcol = region * 64 + ch * 8;
+            if (row < kC) {
+                *ptr = bf16x8_to_f16x8(raw, 1.f);
+                *reinterpret_cast<uint4 *>(p.scr.k16 + (chunk_id * kC + row) * kD + dcol) =
+                    bf16x8_to_f16x8(raw, sm.dec[row]);
+            } else {
+                *reinterpret_cast<uint4 *>(p.scr.wq + (chunk_id * 128 + row) * kD + dcol) =
+                    bf16x8_to_f16x8(raw, sm.gam[row - kC]);
+            }
+        }
+        for (int i = tid; i < 2 * kC * 8; i += 128) {
+            const int region = i >> 9, row = (i >> 3) & 63, ch = i & 7;
+            uint4 *ptr = reinterpret_cast<uint4 *>(sm.v + region * 8192 + sw128_off(row, ch));
+            *ptr = bf16x8_to_f16x8(*ptr, 1.f);
+        }
+        // T = (I + A)^-1, blocked by 16: the diagonal blocks by forward
+        // substitution, then the block diagonals below them in turn,
+        //   T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj   (i > j).
+        // A is strictly lower triangular; T is kept transposed in the upper
+        // triangle (diagonal included) of the same array: T[t][s] at A[s][t].
+        if (tid < kC) {
+            const int bi = tid >> 4, c = tid & 15, o = bi * 16;
+            float x[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                float acc = (t == c) ? 1.f : 0.f;
+#pragma unroll
+                for (int q = 0; q < t; ++q) acc = fmaf(-sm.A[o + t][o + q], x[q], acc);
+                x[t] = (t < c) ? 0.f : acc;
+            }
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                if (t >= c) sm.A[o + c][o + t] = x[t];
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int d = 1; d < 4; ++d) {
+            const int nblk = 4 - d;
+            // Y_ij = sum_k A_ik T_kj for the blocks (i, j = i - d), into T's slot of
+            // the block (held transposed, like T): entry (m, c) at A[16j + c][16i + m]
+            for (int e = tid; e < nblk * 256; e += 128) {
+                const int j = e >> 8, i = j + d, m = (e >> 4) & 15, c = e & 15;
+                float acc = 0.f;
+                for (int k = j; k < i; ++k) {
+                    // T_kj[n][c] sits at A[16j + c][16k + n]; in the diagonal block
+                    // (k == j) the entries n < c of that row are A's, not T's (zero)
+                    const int nlo = k == j ? c : 0;
+#pragma unroll
+                    for (int n = 0; n < 16; n += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(&sm.A[16 * i + m][16 * k + n]);
+                        const float4 t4 = *reinterpret_cast<const float4 *>(&sm.A[16 * j + c][16 * k + n]);
+                        acc = fmaf(a4.x, n >= nlo ? t4.x : 0.f, acc);
+                        acc = fmaf(a4.y, n + 1 >= nlo ? t4.y : 0.f, acc);
+                        acc = fmaf(a4.z, n + 2 >= nlo ? t4.z : 0.f, acc);
+                        acc = fmaf(a4.w, n + 3 >= nlo ? t4.w : 0.f, acc);
+                    }
                 }
+                sm.Y[e] = acc;
             }
-            // Q rows are read: the solve group may now overwrite them
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            for (int i = tid - kC; i < 2 * kC * 8; i += kC) {
-                const int region = i >> 9, row = (i >> 3) & 63, ch = i & 7;
-                uint4 *ptr = reinterpret_cast<uint4 *>(sm.v + region * 8192 + sw128_off(row, ch));
-                *ptr = bf16x8_to_f16x8(*ptr, 1.f);
+            __syncthreads();
+            // T_ij = -T_ii Y_ij
+            for (int e = tid; e < nblk * 256; e += 128) {
+                const int j = e >> 8, i = j + d, r = (e >> 4) & 15, c = e & 15;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(m <= r ? sm.A[16 * i + m][16 * i + r] : 0.f, sm.Y[(j << 8) + (m << 4) + c], acc);
+                sm.A[16 * j + c][16 * i + r] = -acc;
             }
-        } else {
-            // T = (I + A)^-1 by forward substitution, one column per thread.  Row t
-            // of A is zero from column t on and the not-yet-computed entries of the
-            // column are zero, so whole 4-column groups can be read.
-            const int j = tid;
-            float Tc[kC];
+            __syncthreads();
+        }
+        // B operands of the fp16 MMA, K-major rows t over the Q rows of kq:
+        // (T diag(beta g))[t][s] in region 0, (T diag(beta))[t][s] in region 1
+        {
+            const int t = tid & 63;
+            const bool second = tid >= 64;
+            __half *dst = reinterpret_cast<__half *>(sm.kq + (second ? 16384 : 0) + 8192);
 #pragma unroll
-            for (int t = 0; t < kC; ++t) Tc[t] = 0.f;
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t w[4];
 #pragma unroll
-            for (int t = 0; t < kC; ++t) {
-                float a0 = (t == j) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                for (int g4 = 0; g4 < (t + 3) / 4; ++g4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(&sm.A[t][4 * g4]);
-                    a0 = fmaf(-a4.x, Tc[4 * g4], a0);
-                    a1 = fmaf(-a4.y, Tc[4 * g4 + 1], a1);
-                    a2 = fmaf(-a4.z, Tc[4 * g4 + 2], a2);
-                    a3 = fmaf(-a4.w, Tc[4 * g4 + 3], a3);
+                for (int e = 0; e < 8; e += 2) {
+                    const int s0 = ch * 8 + e, s1 = s0 + 1;
+                    const float f0 = second ? sm.beta[s0] : sm.beta[s0] * sm.gam[s0];
+                    const float f1 = second ? sm.beta[s1] : sm.beta[s1] * sm.gam[s1];
+                    const float t0 = s0 <= t ? sm.A[s0][t] : 0.f;
+                    const float t1 = s1 <= t ? sm.A[s1][t] : 0.f;
+                    w[e / 2] = pack_f16x2(t0 * f0, t1 * f1);
                 }
-                Tc[t] = (a0 + a1) + (a2 + a3);
-            }
-            const float bj = sm.beta[j], bgj = sm.beta[j] * sm.gam[j];
-            // wait until the conversion group has read the Q rows
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            __half *b1 = reinterpret_cast<__half *>(sm.kq + 8192);
-            __half *b2 = reinterpret_cast<__half *>(sm.kq + 16384 + 8192);
-#pragma unroll
-            for (int t = 0; t < kC; ++t) {
-                const uint32_t off = sw128_off(t, j >> 3) + (j & 7) * 2;
-                b1[off / 2] = __float2half_rn(Tc[t] * bgj);
-                b2[off / 2] = __float2half_rn(Tc[t] * bj);
+                *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(dst) + sw128_off(t, ch)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
         fence_proxy_async_smem();
@@ -336,7 +380,7 @@ struct __align__(1024) ScanStage {
 
 struct __align__(1024) ScanSmem {
     ScanStage st[2];
-    uint64_t full[2], empty[2], bar_p1, bar_u, bar_o, bar_s16;
+    uint64_t full[2], empty[2], bar_p1, bar_u, bar_d, bar_o, bar_s16, bar_oread;
     uint32_t tmem_base;
     int abort;
 };
@@ -369,8 +413,10 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
         }
         mbar_init(&sm.bar_p1, 1);
         mbar_init(&sm.bar_u, 256);
+        mbar_init(&sm.bar_d, 1);
         mbar_init(&sm.bar_o, 1);
         mbar_init(&sm.bar_s16, 256);
+        mbar_init(&sm.bar_oread, 256);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -414,8 +460,11 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id1 = idesc_f16_f32(128, 128, 0, 0);
-            const uint32_t id2 = idesc_f16_f32(128, 64, 0, 0);
+            // Per chunk, the serial chain is S0 W^T -> U -> U^T K -> S.  The output
+            // half (S0 (gQ)^T + U Pm^T, into columns 64-127 of P1) is issued
+            // beside it; it may only overwrite P1's columns 64-127 once the
+            // previous chunk's output has been read from them.
+            const uint32_t idh = idesc_f16_f32(128, 64, 0, 0);
             const uint32_t id3 = idesc_f16_f32(128, 128, 0, 1);
             int committed = 0;
             for (int c = 0; c < NC; ++c) {
@@ -425,21 +474,34 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
                 if (!mbar_wait(&sm.bar_s16, c & 1, abort, p.dev_err)) break;
                 tc_fence_after();
                 const uint32_t wq = smem_u32(st.wq);
+                // S0 W^T (rows 0-63 of [W; gQ])
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_ts(tmem + kP1, tmem + kS16 + kk * 8,
-                            smem_desc_sw128(wq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id1,
+                            smem_desc_sw128(wq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), idh,
                             kk > 0 ? 1u : 0u);
                 umma_commit(&sm.bar_p1);
+                // S0 (gQ)^T (rows 64-127), reading S16 before the state update rewrites it
+                if (c > 0 && !mbar_wait(&sm.bar_oread, (c - 1) & 1, abort, p.dev_err)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tmem + kP1 + 64, tmem + kS16 + kk * 8,
+                            smem_desc_sw128(wq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32, 16, 1024), idh,
+                            kk > 0 ? 1u : 0u);
                 if (!mbar_wait(&sm.bar_u, c & 1, abort, p.dev_err)) break;
                 tc_fence_after();
                 const uint32_t pm = smem_u32(st.pm), k16 = smem_u32(st.k16);
+                // D = U^T (diag(e^{l_C - l}) K): the state update waits only for this
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    umma_ts(tmem + kP1 + 64, tmem + kU + kk * 8, smem_desc_sw128(pm + kk * 32, 16, 1024), id2, 1u);
+                for (int kk = 0; kk < 4; ++kk)
                     umma_ts(tmem + kDS, tmem + kU + kk * 8, smem_desc_sw128(k16 + kk * 2048, 8192, 1024), id3,
                             kk > 0 ? 1u : 0u);
-                }
+                umma_commit(&sm.bar_d);
+                // O^T += U^T Pm^T
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_ts(tmem + kP1 + 64, tmem + kU + kk * 8, smem_desc_sw128(pm + kk * 32, 16, 1024), idh, 1u);
                 umma_commit(&sm.bar_o);
                 umma_commit(&sm.empty[s]);
                 committed = c + 1;
@@ -506,7 +568,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&sm.bar_u);
             mbar_arrive(&sm.empty[s]);  // done with this stage's U~ and l
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_o, c & 1, abort, p.dev_err))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_d, c & 1, abort, p.dev_err))) {
                 ok = false;
                 break;
             }
@@ -526,14 +588,21 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
                 }
                 tmem_st16(tl + kS16 + 32 * w + 16 * q2, f16w);
             }
-            // O for tokens [32w, 32w+32) must be read before the next chunk's MMA
-            // overwrites it, i.e. before S16 is released
-            uint32_t o[32];
-            tmem_ld32(tl + kP1 + 64 + 32 * w, o);
-            tmem_wait_ld();
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.bar_s16);
+            // O for tokens [32w, 32w+32): read it, then free its columns for the
+            // next chunk's S0 (gQ)^T
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_o, c & 1, abort, p.dev_err))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t o[32];
+            tmem_ld32(tl + kP1 + 64 + 32 * w, o);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_oread);
             // outputs of tokens [32w, 32w+32) of this chunk, column `row`, in groups
             // of 8 tokens whose accumulator loads are issued before their stores
             const int t0 = (p.c_begin + c) * kC + 32 * w;
