@@ -92,6 +92,8 @@ struct __align__(16) Smem {
     KeyTile kt[kMaxKT];
 };
 
+static_assert(sizeof(Smem) + 1024 <= 232448, "attention shared memory exceeds the 227 KB per-block limit");
+
 // Write 32 columns [c0, c0+32) of one output row with the OutMode semantics.
 // The accumulator values are all loaded before any store, so the loads overlap
 // instead of waiting on the stores before them.

@@ -28,6 +28,7 @@
 // value they carry is bounded (unit keys, alpha in (0,1], beta in [0,1]).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -98,6 +99,14 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int t0 = c * kC;
     volatile int *abort = &sm.abort;
 
+    // alpha and beta of the chunk's tokens (tokens past the end act as alpha = 1,
+    // beta = 0): the loads are in flight during the setup below
+    float al = 1.f, be = 0.f;
+    if (tid < kC && t0 + tid < p.L) {
+        const size_t i = ((size_t)b * p.L + t0 + tid) * p.H + h;
+        al = p.alpha[i];
+        be = p.beta[i];
+    }
     if (tid == 0) {
         sm.abort = *reinterpret_cast<volatile int *>(p.dev_err) != 0 ? 1 : 0;
         mbar_init(&sm.bar_tma, 1);
@@ -105,8 +114,10 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(&sm.bar_mma2, 1);
         fence_barrier_init();
     }
+    // 128 columns: [K; Q] K^T in 0-63, later W^T in 0-63 and U~^T in 64-127, so
+    // that four CTAs of this kernel fit one SM's tensor memory
     if (warp == 0) {
-        tmem_alloc(&sm.tmem_base, 256);
+        tmem_alloc(&sm.tmem_base, 128);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -124,16 +135,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tma_load_4d(sm.v, &tmV, 0, h, t0, b, &sm.bar_tma);
         tma_load_4d(sm.v + 8192, &tmV, 64, h, t0, b, &sm.bar_tma);
     }
-    // decay prefix and beta (tokens past the end act as alpha = 1, beta = 0)
+    // decay prefix
     if (tid < kC) {
-        const int t = t0 + tid;
-        float la = 0.f, be = 0.f;
-        if (t < p.L) {
-            const size_t i = ((size_t)b * p.L + t) * p.H + h;
-            la = logf(p.alpha[i]);
-            be = p.beta[i];
-        }
-        float x = la;
+        float x = logf(al);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -205,6 +209,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             for (int j = 0; j < 8; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         }
     }
+    tc_fence_before();  // the TMEM reads above precede the MMA that reuses columns 0-63
     __syncthreads();
 
     if (!*abort) {
@@ -312,7 +317,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     __syncthreads();
 
-    // W^T = K^T (T diag(beta g))^T -> cols 64..127; U~^T = V^T (T diag(beta))^T -> cols 128..191
+    // W^T = K^T (T diag(beta g))^T -> cols 0..63; U~^T = V^T (T diag(beta))^T -> cols 64..127
     if (tid == 0 && !*abort) {
         tc_fence_after();
         const uint32_t idesc = idesc_f16_f32(128, 64, 1, 0);
@@ -320,9 +325,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t b1 = smem_u32(sm.kq + 8192), b2 = smem_u32(sm.kq + 16384 + 8192);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            umma_ss(tmem + 64, smem_desc_sw128(kb + kk * 2048, 16384, 1024), smem_desc_sw128(b1 + kk * 32, 16, 1024),
+            umma_ss(tmem, smem_desc_sw128(kb + kk * 2048, 16384, 1024), smem_desc_sw128(b1 + kk * 32, 16, 1024),
                     idesc, kk > 0 ? 1u : 0u);
-            umma_ss(tmem + 128, smem_desc_sw128(vb + kk * 2048, 8192, 1024), smem_desc_sw128(b2 + kk * 32, 16, 1024),
+            umma_ss(tmem + 64, smem_desc_sw128(vb + kk * 2048, 8192, 1024), smem_desc_sw128(b2 + kk * 32, 16, 1024),
                     idesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sm.bar_mma2);
@@ -334,8 +339,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             uint32_t w[32], u[32];
-            tmem_ld32(tl + 64 + half * 32, w);
-            tmem_ld32(tl + 128 + half * 32, u);
+            tmem_ld32(tl + half * 32, w);
+            tmem_ld32(tl + 64 + half * 32, u);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -349,7 +354,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 128);
     }
 }
 
@@ -363,6 +368,8 @@ struct ScanParams {
     float *S_out;
     const float *gates;
     int out_mode;
+    int out_tma;  // 0: per-token stores; 1: TMA store of fp32 tiles (acc); 2: TMA reduce-add (acc);
+                  // 3: TMA store of bf16 tiles (out)
     float *acc;
     __nv_bfloat16 *out;
     int *dev_err;
@@ -380,10 +387,13 @@ struct __align__(1024) ScanStage {
 
 struct __align__(1024) ScanSmem {
     ScanStage st[2];
-    uint64_t full[2], empty[2], bar_p1, bar_u, bar_d, bar_o, bar_s16, bar_oread;
+    uint8_t ostage[kC * kD * 4];  // one chunk of outputs [token][d_v], fp32 or bf16, for the TMA store
+    uint64_t full[2], empty[2], bar_p1, bar_u, bar_d, bar_o, bar_s16, bar_oread, bar_sfree, bar_sfull;
     uint32_t tmem_base;
     int abort;
 };
+
+static_assert(sizeof(ScanSmem) + 1024 <= 232448, "scan shared memory exceeds the 227 KB per-block limit");
 
 // TMEM columns of the scan
 constexpr uint32_t kP1 = 0;     // [S0 W^T | S0 (gQ)^T]  -> O accumulates on cols 64..127
@@ -396,7 +406,8 @@ constexpr int kScanThreads = 320;  // producer, MMA issuer, 8 math warps
 __global__ void __launch_bounds__(kScanThreads, 1)
 gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant__ CUtensorMap tmK16,
                 const __grid_constant__ CUtensorMap tmPm, const __grid_constant__ CUtensorMap tmUt,
-                const __grid_constant__ CUtensorMap tmEll, const ScanParams p) {
+                const __grid_constant__ CUtensorMap tmEll, const __grid_constant__ CUtensorMap tmOut,
+                const ScanParams p) {
     extern __shared__ uint8_t smem_raw[];
     ScanSmem &sm = *reinterpret_cast<ScanSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -417,6 +428,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
         mbar_init(&sm.bar_o, 1);
         mbar_init(&sm.bar_s16, 256);
         mbar_init(&sm.bar_oread, 256);
+        mbar_init(&sm.bar_sfree, 1);
+        mbar_init(&sm.bar_sfull, 256);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -603,6 +616,46 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_oread);
+            if (p.out_tma) {
+                // the chunk's outputs go through shared memory and one TMA store,
+                // issued by warp 2 once all eight warps have written their tokens
+                const bool elect = warp == 2 && lane == 0;
+                if (elect) {
+                    if (c > 0) bulk_wait_read0();  // the previous chunk's tile has been read
+                    mbar_arrive(&sm.bar_sfree);
+                }
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfree, c & 1, abort, p.dev_err))) {
+                    ok = false;
+                    break;
+                }
+                if (p.out_tma == 3) {
+                    __nv_bfloat16 *st16 = reinterpret_cast<__nv_bfloat16 *>(sm.ostage);
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        st16[(32 * w + t) * kD + row] = __float2bfloat16_rn(gate * __uint_as_float(o[t]));
+                } else {
+                    float *st32 = reinterpret_cast<float *>(sm.ostage);
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) st32[(32 * w + t) * kD + row] = gate * __uint_as_float(o[t]);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar_sfull);
+                if (warp == 2) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, c & 1, abort, p.dev_err))) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        const int tok0 = (p.c_begin + c) * kC;  // rows past L are clipped by the TMA unit
+                        if (p.out_tma == 2)
+                            tma_reduce_add_4d(&tmOut, sm.ostage, 0, h, tok0, b);
+                        else
+                            tma_store_4d(&tmOut, sm.ostage, 0, h, tok0, b);
+                        bulk_commit();
+                    }
+                }
+                continue;
+            }
             // outputs of tokens [32w, 32w+32) of this chunk, column `row`, in groups
             // of 8 tokens whose accumulator loads are issued before their stores
             const int t0 = (p.c_begin + c) * kC + 32 * w;
@@ -631,6 +684,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tmWQ, const __grid_constant_
                 }
             }
         }
+        if (warp == 2 && lane == 0) bulk_wait0();  // stores in flight complete before exit
         if (ok && p.S_out) {
             float *dst = p.S_out + ((size_t)bh * kD + row) * kD + 64 * w;
 #pragma unroll
@@ -690,6 +744,31 @@ bool map_tokens(CUtensorMap *m, const void *base, int H, int L, int B) {
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output tiles of the scan: 4-D view (d_v, H, L, B) of a [B, L, H, 128] fp32 or
+// bf16 tensor, box (128, 1, 64, 1) -- one chunk of one head.
+bool map_out(CUtensorMap *m, const void *base, bool bf16, int H, int L, int B) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || !base) return false;
+    const size_t es = bf16 ? 2 : 4;
+    const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)kD * es, (cuuint64_t)H * kD * es, (cuuint64_t)L * H * kD * es};
+    const cuuint32_t box[4] = {kD, 1, kC, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void *>(base),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// How the scan writes its outputs for an output mode (ScanParams::out_tma), with
+// the tensor map it needs; per-token stores when no TMA form applies.
+int scan_out_tma(CUtensorMap *m, int mode, float *acc, void *out, int H, int L, int B) {
+    memset(m, 0, sizeof(*m));
+    if ((mode == OUT_STORE || mode == OUT_ADD) && map_out(m, acc, false, H, L, B)) return mode == OUT_STORE ? 1 : 2;
+    if (mode == OUT_FINAL_ONLY && map_out(m, out, true, H, L, B)) return 3;
+    memset(m, 0, sizeof(*m));
+    return 0;
 }
 
 class TcGdnImpl : public TcGdn {
@@ -788,6 +867,8 @@ public:
         sp.acc = acc;
         sp.out = static_cast<__nv_bfloat16 *>(out);
         sp.dev_err = dev_err;
+        CUtensorMap mout;
+        sp.out_tma = scan_out_tma(&mout, mode, acc, out, cfg_.H, L, cfg_.B);
         int nlaunch = 0;
         for (int g = 0; g < segs && e == cudaSuccess; ++g) {
             const int c0 = g * per, n = min(per, NC - c0);
@@ -803,7 +884,8 @@ public:
             sp.S_in = g == 0 ? S_in : s_mid_ + (g & 1) * sstride;
             sp.S_out = last ? S_out : s_mid_ + ((g + 1) & 1) * sstride;
             if (e == cudaSuccess)
-                gdn_scan_kernel<<<dim3(cfg_.H, cfg_.B), kScanThreads, scan_smem, s>>>(mwq, mk16, mpm, mut, mell, sp);
+                gdn_scan_kernel<<<dim3(cfg_.H, cfg_.B), kScanThreads, scan_smem, s>>>(mwq, mk16, mpm, mut, mell,
+                                                                                       mout, sp);
             if (e == cudaSuccess) e = cudaGetLastError();
             nlaunch += 2;
             if (last) break;
@@ -979,7 +1061,9 @@ extern "C" HLTA_API hlta_status hlta_gdn_forward_noalloc(int B, int L, int H, co
     sp.acc = nullptr;
     sp.out = static_cast<__nv_bfloat16 *>(out);
     sp.dev_err = dev_err;
-    gdn_scan_kernel<<<dim3(H, B), kScanThreads, sizeof(ScanSmem) + 1024, s>>>(mwq, mk16, mpm, mut, mell, sp);
+    CUtensorMap mout;
+    sp.out_tma = scan_out_tma(&mout, OUT_FINAL_ONLY, nullptr, out, H, L, B);
+    gdn_scan_kernel<<<dim3(H, B), kScanThreads, sizeof(ScanSmem) + 1024, s>>>(mwq, mk16, mpm, mut, mell, mout, sp);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return noalloc_fail(HLTA_ERR_CUDA, cudaGetErrorString(e));
     hlta::set_last_error("");
