@@ -147,33 +147,6 @@ __global__ void ring_append_kernel(RingAppendArgs a, int which) {
 }
 }  // namespace
 
-namespace {
-// Final gated sum when the memory branch ran concurrently into its own
-// accumulator: out = bf16(attention accumulator + memory accumulator).
-__global__ void __launch_bounds__(256) sum_to_bf16_kernel(const float4 *__restrict__ a,
-                                                          const float4 *__restrict__ b, uint4 *__restrict__ out,
-                                                          size_t n8) {
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
-        const float4 a0 = a[2 * i], a1 = a[2 * i + 1], b0 = b[2 * i], b1 = b[2 * i + 1];
-        __nv_bfloat162 r[4] = {__floats2bfloat162_rn(a0.x + b0.x, a0.y + b0.y),
-                               __floats2bfloat162_rn(a0.z + b0.z, a0.w + b0.w),
-                               __floats2bfloat162_rn(a1.x + b1.x, a1.y + b1.y),
-                               __floats2bfloat162_rn(a1.z + b1.z, a1.w + b1.w)};
-        out[i] = *reinterpret_cast<const uint4 *>(r);
-    }
-}
-}  // namespace
-
-cudaError_t launch_sum_to_bf16(const float *a, const float *b, void *out, size_t n, cudaStream_t s) {
-    if (n % 8 != 0) return cudaErrorInvalidValue;
-    const size_t n8 = n / 8;
-    const unsigned blocks = (unsigned)(n8 < (size_t)148 * 16 * 256 ? (n8 + 255) / 256 : 148 * 16);
-    if (n8 == 0) return cudaSuccess;
-    sum_to_bf16_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(a), reinterpret_cast<const float4 *>(b),
-                                              static_cast<uint4 *>(out), n8);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_ring_append(const RingAppendArgs &a, cudaStream_t s) {
     for (int which = 0; which < 2; ++which) {
         const int d = which ? a.d_v : a.d_k;

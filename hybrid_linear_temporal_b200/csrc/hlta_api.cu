@@ -225,8 +225,9 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
     const bool want_attn[2] = {(branches & 1u) != 0, (branches & 2u) != 0};
     // Concurrent schedule: the memory branch (prep kernels and a sequential
     // scan on B*H SMs) runs on the side stream into its own accumulator while
-    // SWA and DSWA run on `s` into theirs; after the join one elementwise pass
-    // writes out = acc + acc2 (the gated sum of all three branches).
+    // the first attention branch runs on `s`; the last attention branch waits
+    // for the memory branch and its epilogue writes out = acc + acc2 + its own
+    // gated output (the gated sum of all three branches).
     const bool overlap = one_shot && (branches & 4u) && (want_attn[0] || want_attn[1]) && h->side &&
                          h->acc2 && h->tc_gdn && h->tc_gdn->covers(nq) && h->tc_attn &&
                          (!want_attn[0] || h->tc_attn->covers(nq, geo[0])) &&
@@ -246,23 +247,24 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
             ps.done(launches);
         }
         CK(cudaEventRecord(h->ev_join, h->side));
-        // both attention branches run on `s` while the memory branch runs
+        // attention on `s` beside the memory branch; the last attention branch
+        // joins it and finishes the output
+        const int n_attn = (want_attn[0] ? 1 : 0) + (want_attn[1] ? 1 : 0);
         int idx = 0;
         for (int br = 0; br < 2; ++br) {
             if (!want_attn[br]) continue;
+            const bool last = idx == n_attn - 1;
+            if (last) CK(cudaStreamWaitEvent(s, h->ev_join, 0));
             ProfScope ps(h, br, s);
             bool done = false;
-            cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, geo[br], in.gates, br,
-                                            idx == 0 ? hlta::OUT_STORE : hlta::OUT_ADD, h->acc, nullptr, out,
-                                            h->dev_err, s, &done);
+            const int mode = last ? (idx == 0 ? hlta::OUT_FINAL_ONLY : hlta::OUT_FINAL) : hlta::OUT_STORE;
+            cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, geo[br], in.gates, br, mode, h->acc,
+                                            last ? h->acc2 : nullptr, out, h->dev_err, s, &done);
             if (e != cudaSuccess || !done)
                 return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
             ps.done(1);
             ++idx;
         }
-        CK(cudaStreamWaitEvent(s, h->ev_join, 0));
-        CK(hlta::launch_sum_to_bf16(h->acc, h->acc2, out, (size_t)c.B * nq * c.H * c.d_v, s));
-        if (h->prof) h->prof_launches += 1;
         return HLTA_OK;
     }
     for (int idx = 0; idx < n; ++idx) {

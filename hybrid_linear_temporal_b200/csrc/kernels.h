@@ -68,7 +68,5 @@ void set_last_error(const char *msg);
 cudaError_t launch_attn_simt(const AttnSimtArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_gdn_recurrent(const GdnRecArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_ring_append(const RingAppendArgs &a, cudaStream_t s);
-// out[i] = bf16(a[i] + b[i]) for i < n (n a multiple of 8, pointers 16-byte aligned).
-cudaError_t launch_sum_to_bf16(const float *a, const float *b, void *out, size_t n, cudaStream_t s);
 
 }  // namespace hlta
