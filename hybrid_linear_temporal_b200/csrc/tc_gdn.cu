@@ -75,7 +75,6 @@ struct __align__(1024) PrepSmem {
     uint8_t kq[32768];
     uint8_t v[16384];    // 2 regions x 64 rows of V
     float A[kC][kC + 4];  // rows padded to 16 bytes; T^T is built in the upper triangle
-    float Y[3 * 256];     // block products of the triangular inverse
     float ell[kC], beta[kC], gam[kC], dec[kC];
     uint64_t bar_tma, bar_mma1, bar_mma2;
     uint32_t tmem_base;
@@ -255,39 +254,65 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (t >= c) sm.A[o + c][o + t] = x[t];
         }
         __syncthreads();
+        // Block diagonal d: one thread per column c of each block (i, j = i - d).
+        // It forms y = sum_k A_ik T_kj[:, c] (16 values), then
+        // T_ij[:, c] = -T_ii y, with sixteen independent accumulators each time.
 #pragma unroll 1
         for (int d = 1; d < 4; ++d) {
-            const int nblk = 4 - d;
-            // Y_ij = sum_k A_ik T_kj for the blocks (i, j = i - d), into T's slot of
-            // the block (held transposed, like T): entry (m, c) at A[16j + c][16i + m]
-            for (int e = tid; e < nblk * 256; e += 128) {
-                const int j = e >> 8, i = j + d, m = (e >> 4) & 15, c = e & 15;
-                float acc = 0.f;
+            if (tid < (4 - d) * 16) {
+                const int j = tid >> 4, i = j + d, c = tid & 15;
+                float y[16];
+#pragma unroll
+                for (int mrow = 0; mrow < 16; ++mrow) y[mrow] = 0.f;
                 for (int k = j; k < i; ++k) {
                     // T_kj[n][c] sits at A[16j + c][16k + n]; in the diagonal block
                     // (k == j) the entries n < c of that row are A's, not T's (zero)
-                    const int nlo = k == j ? c : 0;
+                    float tc[16];
 #pragma unroll
                     for (int n = 0; n < 16; n += 4) {
-                        const float4 a4 = *reinterpret_cast<const float4 *>(&sm.A[16 * i + m][16 * k + n]);
                         const float4 t4 = *reinterpret_cast<const float4 *>(&sm.A[16 * j + c][16 * k + n]);
-                        acc = fmaf(a4.x, n >= nlo ? t4.x : 0.f, acc);
-                        acc = fmaf(a4.y, n + 1 >= nlo ? t4.y : 0.f, acc);
-                        acc = fmaf(a4.z, n + 2 >= nlo ? t4.z : 0.f, acc);
-                        acc = fmaf(a4.w, n + 3 >= nlo ? t4.w : 0.f, acc);
+                        tc[n] = t4.x;
+                        tc[n + 1] = t4.y;
+                        tc[n + 2] = t4.z;
+                        tc[n + 3] = t4.w;
+                    }
+                    if (k == j) {
+#pragma unroll
+                        for (int n = 0; n < 16; ++n)
+                            if (n < c) tc[n] = 0.f;
+                    }
+#pragma unroll
+                    for (int mrow = 0; mrow < 16; ++mrow) {
+#pragma unroll
+                        for (int n = 0; n < 16; n += 4) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(&sm.A[16 * i + mrow][16 * k + n]);
+                            y[mrow] = fmaf(a4.x, tc[n], y[mrow]);
+                            y[mrow] = fmaf(a4.y, tc[n + 1], y[mrow]);
+                            y[mrow] = fmaf(a4.z, tc[n + 2], y[mrow]);
+                            y[mrow] = fmaf(a4.w, tc[n + 3], y[mrow]);
+                        }
                     }
                 }
-                sm.Y[e] = acc;
-            }
-            __syncthreads();
-            // T_ij = -T_ii Y_ij
-            for (int e = tid; e < nblk * 256; e += 128) {
-                const int j = e >> 8, i = j + d, r = (e >> 4) & 15, c = e & 15;
-                float acc = 0.f;
+                // T_ij[r][c] = -sum_{m <= r} T_ii[r][m] y[m]; T_ii[r][m] sits at A[16i + m][16i + r]
+                float tr[16];
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(m <= r ? sm.A[16 * i + m][16 * i + r] : 0.f, sm.Y[(j << 8) + (m << 4) + c], acc);
-                sm.A[16 * j + c][16 * i + r] = -acc;
+                for (int r = 0; r < 16; ++r) tr[r] = 0.f;
+#pragma unroll
+                for (int mrow = 0; mrow < 16; ++mrow) {
+#pragma unroll
+                    for (int r = 0; r < 16; r += 4) {
+                        if (r + 3 < mrow) continue;
+                        const float4 t4 = *reinterpret_cast<const float4 *>(&sm.A[16 * i + mrow][16 * i + r]);
+                        if (r >= mrow) tr[r] = fmaf(t4.x, y[mrow], tr[r]);
+                        if (r + 1 >= mrow) tr[r + 1] = fmaf(t4.y, y[mrow], tr[r + 1]);
+                        if (r + 2 >= mrow) tr[r + 2] = fmaf(t4.z, y[mrow], tr[r + 2]);
+                        if (r + 3 >= mrow) tr[r + 3] = fmaf(t4.w, y[mrow], tr[r + 3]);
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 16; r += 4)
+                    *reinterpret_cast<float4 *>(&sm.A[16 * j + c][16 * i + r]) =
+                        make_float4(-tr[r], -tr[r + 1], -tr[r + 2], -tr[r + 3]);
             }
             __syncthreads();
         }
