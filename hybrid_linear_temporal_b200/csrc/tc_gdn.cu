@@ -923,7 +923,7 @@ public:
 
 private:
     hlta_config cfg_;
-    static constexpr int kSegs = 8;
+    static constexpr int kSegs = 4;
     int max_nc_;
     void *base_ = nullptr;
     float *s_mid_ = nullptr;
