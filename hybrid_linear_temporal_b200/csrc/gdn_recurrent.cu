@@ -1,8 +1,9 @@
 // gdn_recurrent.cu -- token-by-token gated delta memory (CUDA cores, fp32 state).
 //
-// Kairos paper, section 2.2.1 (Eq. (2)-(6), step 4), decayed-retrieval form:
-//   v_old = alpha_t S_{t-1} k_t,  u_t = beta_t (v_t - v_old),
-//   S_t = alpha_t S_{t-1} + u_t k_t^T,  o_t = S_t q_t.
+// Kairos paper, section 2.2.1 (Eq. (2)-(6), step 4):
+//   v_old = alpha_t S_{t-1} k_t (decayed retrieval, the default form) or
+//   v_old = S_{t-1} k_t (Eq. (2)/(6) as printed, HLTA_GDN_PAGES),
+//   u_t = beta_t (v_t - v_old),  S_t = alpha_t S_{t-1} + u_t k_t^T,  o_t = S_t q_t.
 // The rows of S (value dimension) evolve independently, so each warp owns a
 // few rows across all d_k columns (d_k/32 columns per lane, vectorised loads)
 // and the grid splits d_v across CTAs.  Per token the warp needs S k, S q and
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(kWarps * 32) gdn_recurrent_kernel(GdnRecArgs a
         for (int j = 0; j < CPL; ++j) S[r][j] = a.S_in ? a.S_in[sbase + (size_t)r * DK + j] : 0.f;
 
     const float gate = a.gates[h * 3 + 2];
+    const bool printed = a.form == HLTA_GDN_PAGES;
     TokenIn<T, DK, RPW> cur, nxt;
     if (a.n > 0) load_token<T, DK, RPW>(cur, a, ((size_t)b * a.n) * a.H + h, lane, row0);
     for (int t = 0; t < a.n; ++t) {
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(kWarps * 32) gdn_recurrent_kernel(GdnRecArgs a
         float outv = 0.f;
 #pragma unroll
         for (int r = 0; r < RPW; ++r) {
-            const float u = cur.be * (cur.v[r] - cur.al * red[2 * r]);
+            const float u = cur.be * (cur.v[r] - (printed ? 1.f : cur.al) * red[2 * r]);
 #pragma unroll
             for (int j = 0; j < CPL; ++j) S[r][j] = fmaf(cur.al, S[r][j], u * cur.k[j]);
             const float o_r = fmaf(cur.al, red[2 * r + 1], u * kq);

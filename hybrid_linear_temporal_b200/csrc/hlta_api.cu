@@ -134,6 +134,8 @@ hlta_status check_config(const hlta_config *c) {
         return fail(HLTA_ERR_INVALID_ARG, "dtype must be HLTA_BF16 or HLTA_FP32");
     if (c->max_seq_len < 1) return fail(HLTA_ERR_INVALID_ARG, "max_seq_len must be >= 1");
     if (c->max_stream_tokens < 0) return fail(HLTA_ERR_INVALID_ARG, "max_stream_tokens must be >= 0");
+    if (c->gdn_form != HLTA_GDN_DECAYED && c->gdn_form != HLTA_GDN_PAGES)
+        return fail(HLTA_ERR_INVALID_ARG, "gdn_form must be HLTA_GDN_DECAYED or HLTA_GDN_PAGES");
     if ((c->d_k != 64 && c->d_k != 128) || (c->d_v != 64 && c->d_v != 128))
         return fail(HLTA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128");
     if (c->chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64");
@@ -332,6 +334,7 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
                 a.out_mode = mode;
                 a.acc = h->acc;
                 a.out = out;
+                a.form = c.gdn_form;
                 CK(hlta::launch_gdn_recurrent(a, bf16, s));
             }
         }

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "hlta.h"
+
 namespace hlta {
 
 // How a branch kernel writes its gated output g*o into the layer output.
@@ -53,6 +55,7 @@ struct GdnRecArgs {
     int out_mode;
     float *acc;
     void *out;
+    int form;  // HLTA_GDN_DECAYED / HLTA_GDN_PAGES: what the retrieval reads
 };
 
 struct RingAppendArgs {

@@ -9,6 +9,9 @@
 //   T = (I + A)^-1,  W = T diag(beta g) K,  U~ = T diag(beta) V,  U = U~ - W S0^T
 //   O = diag(g) Q S0^T + Pm U,                Pm_ts = e^{l_t-l_s} q_t.k_s (s <= t)
 //   S_C = g_C S0 + U^T diag(e^{l_C-l}) K.
+// The update form printed as Eq. (2)/(6), u_t = beta_t (v_t - S_{t-1} k_t), is the
+// same system with l_t replaced by l_{t-1} in A's rows and in W's factors
+// (HLTA_GDN_PAGES).
 // Two kernels:
 //   gdn_prep_kernel  (one CTA per chunk, all chunks in parallel): [K;Q] K^T on
 //       tcgen05 (bf16), the decay masks, T by blocked forward substitution on
@@ -64,6 +67,7 @@ struct PrepParams {
     const float *alpha, *beta;  // [B, L, H]
     int L, H, NC;
     int c_begin;                // first chunk of this launch (blockIdx.x is relative)
+    int form;                   // HLTA_GDN_DECAYED / HLTA_GDN_PAGES
     GdnScratch scr;
     int *dev_err;
 };
@@ -76,6 +80,7 @@ struct __align__(1024) PrepSmem {
     uint8_t v[16384];    // 2 regions x 64 rows of V
     float A[kC][kC + 4];  // rows padded to 16 bytes; T^T is built in the upper triangle
     float ell[kC], beta[kC], gam[kC], dec[kC];
+    float ellr[kC], gamr[kC];  // log-decay / decay that token t's retrieval sees (see below)
     uint64_t bar_tma, bar_mma1, bar_mma2;
     uint32_t tmem_base;
     int abort;
@@ -151,6 +156,13 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (tid < kC) {
         sm.gam[tid] = expf(sm.ell[tid]);
         sm.dec[tid] = expf(sm.ell[kC - 1] - sm.ell[tid]);
+        // The retrieval of token t reads alpha_t S_{t-1} (decayed form: l_t) or
+        // S_{t-1} (the printed Eq. (2)/(6): l_{t-1}, 0 for the chunk's first
+        // token).  Only A's rows and W's factors depend on it; with
+        // beta'_t = beta_t / alpha_t the printed form is the decayed form, and
+        // forming e^{l_{t-1} - l_s} directly keeps every factor <= 1.
+        sm.ellr[tid] = p.form == HLTA_GDN_PAGES ? (tid == 0 ? 0.f : sm.ell[tid - 1]) : sm.ell[tid];
+        sm.gamr[tid] = expf(sm.ellr[tid]);
         p.scr.ell[chunk_id * 2 * kC + tid] = sm.ell[tid];
         p.scr.ell[chunk_id * 2 * kC + kC + tid] = sm.dec[tid];
     }
@@ -180,7 +192,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_wait_ld();
         if (tid < kC) {
             const int t = tid;
-            const float lt = sm.ell[t], bt = sm.beta[t];
+            const float lt = sm.ellr[t], bt = sm.beta[t];
 #pragma unroll
             for (int s = 0; s < kC; s += 4) {
                 float a[4];
@@ -328,8 +340,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     const int s0 = ch * 8 + e, s1 = s0 + 1;
-                    const float f0 = second ? sm.beta[s0] : sm.beta[s0] * sm.gam[s0];
-                    const float f1 = second ? sm.beta[s1] : sm.beta[s1] * sm.gam[s1];
+                    const float f0 = second ? sm.beta[s0] : sm.beta[s0] * sm.gamr[s0];
+                    const float f1 = second ? sm.beta[s1] : sm.beta[s1] * sm.gamr[s1];
                     const float t0 = s0 <= t ? sm.A[s0][t] : 0.f;
                     const float t1 = s1 <= t ? sm.A[s1][t] : 0.f;
                     w[e / 2] = pack_f16x2(t0 * f0, t1 * f1);
@@ -881,6 +893,7 @@ public:
         pp.L = L;
         pp.H = cfg_.H;
         pp.NC = NC;
+        pp.form = cfg_.gdn_form;
         pp.scr = scr;
         pp.dev_err = dev_err;
         ScanParams sp;
@@ -1070,6 +1083,7 @@ extern "C" HLTA_API hlta_status hlta_gdn_forward_noalloc(int B, int L, int H, co
     pp.H = H;
     pp.NC = NC;
     pp.c_begin = 0;
+    pp.form = HLTA_GDN_DECAYED;
     pp.scr = scr;
     pp.dev_err = dev_err;
     gdn_prep_kernel<<<dim3(NC, H, B), 128, sizeof(PrepSmem) + 1024, s>>>(mq, mk, mv, pp);

@@ -74,6 +74,17 @@ enum {
     HLTA_BRANCH_ALL = 7
 };
 
+/* Form of the memory update (hlta_config.gdn_form).  Both share
+ *   S_t = alpha_t S_{t-1} + u_t k_t^T,  o_t = S_t q_t  (section 2.2.1, Eq. (5), step 4)
+ * and differ in what the retrieval of Eq. (2) reads:
+ *   HLTA_GDN_DECAYED  u_t = beta_t (v_t - alpha_t S_{t-1} k_t): the decayed state, i.e.
+ *                     S_t = alpha_t S_{t-1}(I - beta_t k_t k_t^T) + beta_t v_t k_t^T.
+ *                     The layer's fixed form and the default.
+ *   HLTA_GDN_PAGES    u_t = beta_t (v_t - S_{t-1} k_t): Eq. (2) and Eq. (6) as printed.
+ *                     Contractive as well, with factor max(alpha, |alpha - beta|) < 1 along
+ *                     a unit k_t. */
+enum { HLTA_GDN_DECAYED = 0, HLTA_GDN_PAGES = 1 };
+
 /* Layer configuration, fixed for the life of a handle. */
 typedef struct {
     int B;                 /* batch, >= 1 */
@@ -88,6 +99,7 @@ typedef struct {
     int dtype;             /* hlta_dtype of q, k, v and out */
     int max_seq_len;       /* largest L accepted by hlta_forward (>= 1) */
     int max_stream_tokens; /* largest n of hlta_stream_step; 0 disables streaming */
+    int gdn_form;          /* HLTA_GDN_DECAYED (0) or HLTA_GDN_PAGES (1) */
 } hlta_config;
 
 typedef struct hlta_handle hlta_handle;

@@ -156,11 +156,13 @@ def gdn_chunked(q, k, v, alpha, beta, chunk: int, S0=None):
     return out, S
 
 
-def forward(inp, S0=None, branches=("swa", "dswa", "gdn")):
+def forward(inp, S0=None, branches=("swa", "dswa", "gdn"), variant=0):
     """The whole layer: out = g_swa[h]*SWA + g_dswa[h]*DSWA + g_gdn[h]*GDN.
 
     inp: a ``workloads.Inputs``.  The branch combination (a per-head weighted
-    sum) is the specification's; the pages leave it open.
+    sum) is the specification's; the pages leave it open.  variant selects the
+    memory update form of ``gdn`` (0: decayed retrieval, 1: Eq. (2)/(6) as
+    printed).
     Returns dict with 'out' [B,L,H,d_v], per-branch outputs and 'S'.
     """
     wl = inp.wl
@@ -173,7 +175,7 @@ def forward(inp, S0=None, branches=("swa", "dswa", "gdn")):
     if "dswa" in branches:
         res["dswa"] = attention("dswa", inp.q, inp.k, inp.v, wl.P, wl.dilation, wl.dswa_window)
         total = total + g[None, None, :, 1, None] * res["dswa"]
-    o, S = gdn(inp.q, inp.k, inp.v, inp.alpha, inp.beta, S0)
+    o, S = gdn(inp.q, inp.k, inp.v, inp.alpha, inp.beta, S0, variant=variant)
     res["S"] = S
     if "gdn" in branches:
         res["gdn"] = o

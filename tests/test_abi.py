@@ -37,7 +37,8 @@ def test_version(lib):
 
 def _cfg(**kw):
     base = dict(B=1, H=2, d_k=64, d_v=64, tokens_per_frame=4, swa_window=8, dswa_window=8,
-                dswa_dilation=2, chunk=64, dtype=binding.BF16, max_seq_len=128, max_stream_tokens=0)
+                dswa_dilation=2, chunk=64, dtype=binding.BF16, max_seq_len=128, max_stream_tokens=0,
+                gdn_form=binding.GDN_DECAYED)
     base.update(kw)
     return binding.Config(*[base[n] for n, _ in binding.Config._fields_])
 
@@ -47,6 +48,7 @@ def _cfg(**kw):
     ("tokens_per_frame", 0, binding.ERR_INVALID_ARG), ("swa_window", 0, binding.ERR_INVALID_ARG),
     ("dswa_dilation", 0, binding.ERR_INVALID_ARG), ("dtype", 5, binding.ERR_INVALID_ARG),
     ("max_seq_len", 0, binding.ERR_INVALID_ARG), ("max_stream_tokens", -2, binding.ERR_INVALID_ARG),
+    ("gdn_form", 2, binding.ERR_INVALID_ARG), ("gdn_form", -1, binding.ERR_INVALID_ARG),
     ("d_k", 96, binding.ERR_UNSUPPORTED), ("chunk", 32, binding.ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_config_before_device(lib, field, value, status):

@@ -33,10 +33,10 @@ def layer_for(wl, **kw):
 
 
 def full_compare(torch_cuda, wl, seed=0, alpha_mode="default", q_scale=1.0, S0=None,
-                 branches=("swa", "dswa", "gdn")):
+                 branches=("swa", "dswa", "gdn"), gdn_form=0):
     inp = make_inputs(wl, seed=seed, alpha_mode=alpha_mode, q_scale=q_scale)
-    ref = oracle.forward(inp, S0=S0, branches=branches)
-    layer = layer_for(wl)
+    ref = oracle.forward(inp, S0=S0, branches=branches, variant=gdn_form)
+    layer = layer_for(wl, gdn_form=gdn_form)
     dev = to_device(inp)
     S0_dev = None if S0 is None else torch_cuda.from_numpy(S0.astype(np.float32)).cuda()
     mask = sum(1 << i for i, n in enumerate(("swa", "dswa", "gdn")) if n in branches)
@@ -57,6 +57,23 @@ def full_compare(torch_cuda, wl, seed=0, alpha_mode="default", q_scale=1.0, S0=N
 
 def test_tiny_fp32(torch_cuda):
     full_compare(torch_cuda, WORKLOADS["tiny_fp32"])
+
+
+def test_pages_form_tiny_fp32(torch_cuda):
+    """The memory update as Eq. (2)/(6) print it (token recurrence on CUDA cores)."""
+    full_compare(torch_cuda, WORKLOADS["tiny_fp32"], gdn_form=1)
+
+
+def test_pages_form_clip_4k_bf16(torch_cuda):
+    """The printed update form through the chunked tensor-core path."""
+    full_compare(torch_cuda, WORKLOADS["clip_4k"], gdn_form=1)
+
+
+def test_pages_form_long_memory_bf16(torch_cuda):
+    """The printed form with alpha ~ 0.98 (long memory) on a ragged length.  The
+    default inputs already have alpha ~ 0.1, where beta/alpha is large."""
+    wl = WORKLOADS["clip_4k"].with_(L=1000, H=4)
+    full_compare(torch_cuda, wl, seed=3, alpha_mode="slow", branches=("gdn",), gdn_form=1)
 
 
 def test_clip_4k_bf16(torch_cuda):
