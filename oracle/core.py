@@ -39,6 +39,9 @@ def _load():
         lib.oracle_attention.argtypes = [i, i, i, i, i, i, i, i, i, vp, vp, vp, i, l,
                                          ctypes.POINTER(ctypes.c_longlong), l, dp]
         lib.oracle_attention.restype = i
+        lib.oracle_attention_centred.argtypes = [i, ctypes.c_double, i, i, i, i, i, i, i, i, vp, vp, vp, i,
+                                                 l, ctypes.POINTER(ctypes.c_longlong), l, dp]
+        lib.oracle_attention_centred.restype = i
         lib.oracle_gdn.argtypes = [i, i, i, i, i, vp, vp, vp, i, fp, fp, dp, dp, dp, i, i]
         lib.oracle_gdn.restype = i
         lib.oracle_gdn_chunked.argtypes = [i, i, i, i, i, vp, vp, vp, i, fp, fp, dp, dp, dp, i]
@@ -75,13 +78,17 @@ def dswa_span(P: int, dilation: int, w: int) -> int:
 
 
 def attention_rows(kind: str, q, k, v, P: int, dilation: int, w: int, rows=None,
-                   span: int | None = None) -> np.ndarray:
+                   span: int | None = None, centred: bool = False,
+                   rope_base: float = 0.0) -> np.ndarray:
     """Softmax attention rows under the SWA ("swa") or DSWA ("dswa") mask.
 
     q, k: [B, L, H, d_k], v: [B, L, H, d_v] (uint16 bf16 bits or float32).
     rows: int64 row ids (b*L + t)*H + h, or None for all rows.  Returns
     [nrows, d_v] float64 (or [B, L, H, d_v] when rows is None).
-    span: None chooses a provable bound; -1 examines every key j <= i.
+    span: None chooses a provable bound; -1 examines every key.
+    centred: the centred window |r(i) - r(j)| <= w // 2 instead of the causal
+    one; rope_base > 0 rotates q and k by their token positions first
+    (oracle_attention_centred in hlta_oracle.c).
     """
     lib = _load()
     q, dt = _tensor(q)
@@ -92,7 +99,10 @@ def attention_rows(kind: str, q, k, v, P: int, dilation: int, w: int, rows=None,
     dv = v.shape[-1]
     kind_i = {"swa": 0, "dswa": 1}[kind]
     if span is None:
-        span = w - 1 if kind == "swa" else dswa_span(P, dilation, w)
+        if centred:
+            span = w // 2 if kind == "swa" else dswa_span(P, dilation, w // 2)
+        else:
+            span = w - 1 if kind == "swa" else dswa_span(P, dilation, w)
     if rows is None:
         n = B * L * H
         rp = None
@@ -102,16 +112,23 @@ def attention_rows(kind: str, q, k, v, P: int, dilation: int, w: int, rows=None,
         n = rows.size
         rp = rows.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong))
         out = np.empty((n, dv), dtype=np.float64)
-    rc = lib.oracle_attention(kind_i, B, L, H, dk, dv, P, dilation, w,
-                              q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, n, rp, span,
-                              _dptr(out))
+    if centred or rope_base > 0.0:
+        if not centred:
+            raise ValueError("rotary embedding is provided with the centred window only")
+        rc = lib.oracle_attention_centred(kind_i, float(rope_base), B, L, H, dk, dv, P, dilation, w,
+                                          q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, n, rp, span,
+                                          _dptr(out))
+    else:
+        rc = lib.oracle_attention(kind_i, B, L, H, dk, dv, P, dilation, w,
+                                  q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, n, rp, span,
+                                  _dptr(out))
     if rc != 0:
         raise ValueError("oracle_attention: bad arguments")
     return out
 
 
-def attention(kind, q, k, v, P, dilation, w, span=None):
-    return attention_rows(kind, q, k, v, P, dilation, w, None, span)
+def attention(kind, q, k, v, P, dilation, w, span=None, centred=False, rope_base=0.0):
+    return attention_rows(kind, q, k, v, P, dilation, w, None, span, centred, rope_base)
 
 
 def _gdn_common(q, k, v, alpha, beta, S0):

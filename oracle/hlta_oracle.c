@@ -19,6 +19,10 @@
  *   oracle_attention  -- section 2.2.2, Eq. (7) (SWA) and Eq. (8) (DSWA), with
  *                        the causal window and residue-class dilation readings
  *                        documented beside each predicate below.
+ *   oracle_attention_centred -- the same with the centred window Eq. (7) prints
+ *                        (the diffusion in-clip reading) and, optionally, rotary
+ *                        position embedding on q and k (the pages name RoPE on the
+ *                        sliding-window blocks; the rotation below is a reading).
  *   oracle_gdn        -- section 2.2.1, steps 2-4 (Eq. (2)-(6)) and the output
  *                        o_t = S_t q_t.
  *   oracle_gdn_chunked-- the same recurrence regrouped into chunks (a
@@ -78,6 +82,32 @@ static inline int dswa_in_window(long i, long j, long P, long dil, long w) {
     return dr >= 0 && dr < w;
 }
 
+/* Centred reading of Eq. (7): key j is admitted iff |i - j| <= floor(w/2) (for
+ * DSWA: in the same residue class and |r(i) - r(j)| <= floor(w/2)). */
+static inline int swa_in_centred(long i, long j, long w) {
+    long d = i - j;
+    return (d < 0 ? -d : d) <= w / 2;
+}
+
+static inline int dswa_in_centred(long i, long j, long P, long dil, long w) {
+    long fi = i / P, fj = j / P;
+    if ((fi - fj) % dil != 0) return 0;
+    long dr = rearranged_pos(i, P, dil) - rearranged_pos(j, P, dil);
+    return (dr < 0 ? -dr : dr) <= w / 2;
+}
+
+/* Rotary position embedding (reading): for token position t and channel pair
+ * (2m, 2m+1), m < d/2, rotate (x_2m, x_2m+1) by the angle t * base^(-2m/d). */
+static void rope_rotate(double *x, int d, long t, double base) {
+    for (int m = 0; 2 * m + 1 < d; ++m) {
+        double theta = (double)t * pow(base, -2.0 * m / (double)d);
+        double c = cos(theta), sn = sin(theta);
+        double a = x[2 * m], b = x[2 * m + 1];
+        x[2 * m] = a * c - b * sn;
+        x[2 * m + 1] = a * sn + b * c;
+    }
+}
+
 /*
  * oracle_attention: softmax attention rows under the SWA (kind 0) or DSWA
  * (kind 1) mask.
@@ -92,18 +122,20 @@ static inline int dswa_in_window(long i, long j, long P, long dil, long w) {
  * at least as large as the farthest admitted key gives the same result.
  * Returns 0, or -1 on bad arguments.
  */
-int oracle_attention(int kind, int B, int L, int H, int d_k, int d_v, int P, int dil, int w,
-                     const void *q, const void *k, const void *v, int dt, long nrows,
-                     const long long *rows, long span, double *out) {
+static int attention_core(int kind, int centred, double rope_base, int B, int L, int H, int d_k,
+                          int d_v, int P, int dil, int w, const void *q, const void *k, const void *v,
+                          int dt, long nrows, const long long *rows, long span, double *out) {
     if (B <= 0 || L <= 0 || H <= 0 || d_k <= 0 || d_v <= 0 || P <= 0 || dil <= 0 || w <= 0)
         return -1;
     if (kind != 0 && kind != 1) return -1;
+    if (rope_base < 0.0 || (rope_base > 0.0 && d_k % 2 != 0)) return -1;
     const double scale = 1.0 / sqrt((double)d_k);
 
 #pragma omp parallel
     {
         double *logit = (double *)malloc(sizeof(double) * (size_t)L);
         double *qi = (double *)malloc(sizeof(double) * (size_t)d_k);
+        double *kj = (double *)malloc(sizeof(double) * (size_t)d_k);
 #pragma omp for schedule(dynamic, 16)
         for (long r = 0; r < nrows; ++r) {
             long long id = rows ? rows[r] : (long long)r;
@@ -112,17 +144,25 @@ int oracle_attention(int kind, int B, int L, int H, int d_k, int d_v, int P, int
             long b = (long)(id / ((long long)H * L));
             size_t qoff = (((size_t)b * L + t) * H + h) * d_k;
             for (int c = 0; c < d_k; ++c) qi[c] = load_elem(q, dt, qoff + c);
+            if (rope_base > 0.0) rope_rotate(qi, d_k, t, rope_base);
             long lo = (span < 0 || t - span < 0) ? 0 : t - span;
+            long hi = !centred ? t : ((span < 0 || t + span > L - 1) ? L - 1 : t + span);
             double m = -INFINITY;
-            for (long j = lo; j <= t; ++j) {
-                int in = kind == 0 ? swa_in_window(t, j, w) : dswa_in_window(t, j, P, dil, w);
+            for (long j = lo; j <= hi; ++j) {
+                int in;
+                if (centred)
+                    in = kind == 0 ? swa_in_centred(t, j, w) : dswa_in_centred(t, j, P, dil, w);
+                else
+                    in = kind == 0 ? swa_in_window(t, j, w) : dswa_in_window(t, j, P, dil, w);
                 if (!in) {
                     logit[j] = NAN; /* marks a masked key */
                     continue;
                 }
                 size_t koff = (((size_t)b * L + j) * H + h) * d_k;
+                for (int c = 0; c < d_k; ++c) kj[c] = load_elem(k, dt, koff + c);
+                if (rope_base > 0.0) rope_rotate(kj, d_k, j, rope_base);
                 double s = 0.0;
-                for (int c = 0; c < d_k; ++c) s += qi[c] * load_elem(k, dt, koff + c);
+                for (int c = 0; c < d_k; ++c) s += qi[c] * kj[c];
                 s *= scale;
                 logit[j] = s;
                 if (s > m) m = s;
@@ -130,7 +170,7 @@ int oracle_attention(int kind, int B, int L, int H, int d_k, int d_v, int P, int
             double *o = out + (size_t)r * d_v;
             for (int c = 0; c < d_v; ++c) o[c] = 0.0;
             double denom = 0.0;
-            for (long j = lo; j <= t; ++j) {
+            for (long j = lo; j <= hi; ++j) {
                 if (isnan(logit[j])) continue;
                 double p = exp(logit[j] - m);
                 denom += p;
@@ -141,8 +181,29 @@ int oracle_attention(int kind, int B, int L, int H, int d_k, int d_v, int P, int
         }
         free(logit);
         free(qi);
+        free(kj);
     }
     return 0;
+}
+
+int oracle_attention(int kind, int B, int L, int H, int d_k, int d_v, int P, int dil, int w,
+                     const void *q, const void *k, const void *v, int dt, long nrows,
+                     const long long *rows, long span, double *out) {
+    return attention_core(kind, 0, 0.0, B, L, H, d_k, d_v, P, dil, w, q, k, v, dt, nrows, rows, span,
+                          out);
+}
+
+/*
+ * oracle_attention_centred: as oracle_attention with the centred window
+ * (|r(i) - r(j)| <= floor(w/2), see the predicates above) and, when
+ * rope_base > 0, q and k rotated by rope_rotate at their token positions before
+ * the dot product.  span bounds |i - j| from above (< 0: every key).
+ */
+int oracle_attention_centred(int kind, double rope_base, int B, int L, int H, int d_k, int d_v, int P,
+                             int dil, int w, const void *q, const void *k, const void *v, int dt,
+                             long nrows, const long long *rows, long span, double *out) {
+    return attention_core(kind, 1, rope_base, B, L, H, d_k, d_v, P, dil, w, q, k, v, dt, nrows, rows,
+                          span, out);
 }
 
 /* ------------------------------------------------------------------------ */

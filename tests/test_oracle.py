@@ -457,3 +457,87 @@ def test_inputs_deterministic_and_distributed():
     assert np.all(np.abs(qn - 1) < 1e-2)
     assert 0.1 < a.alpha.mean() < 0.2 and a.alpha.max() < 1
     assert 0.3 < a.beta.mean() < 0.7
+
+
+# --------------------------------------------------------------------------
+# Centred windows and rotary embedding (the bidirectional reading of Eq. (7),
+# RoPE on the sliding-window blocks)
+# --------------------------------------------------------------------------
+
+def _rand_qkv(B, L, H, d, seed=0):
+    rng = np.random.default_rng(seed)
+    return tuple(rng.standard_normal((B, L, H, d)).astype(np.float32) for _ in range(3))
+
+
+def _masked_softmax_attention(q, k, v, admit):
+    """Dense softmax attention with an explicit [L, L] admission matrix
+    (numpy library routines; a check independent of the oracle's loops)."""
+    s = np.einsum("blhd,bmhd->bhlm", q.astype(np.float64), k.astype(np.float64)) / math.sqrt(q.shape[-1])
+    s = np.where(admit[None, None], s, -np.inf)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    return np.einsum("bhlm,bmhd->blhd", p, v.astype(np.float64))
+
+
+def test_centred_window_wider_than_sequence_is_bidirectional_attention():
+    q, k, v = _rand_qkv(1, 37, 2, 8)
+    got = oracle.attention("swa", q, k, v, 1, 1, 1000, centred=True)
+    want = _masked_softmax_attention(q, k, v, np.ones((37, 37), bool))
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-13)
+
+
+def test_centred_window_band_matches_explicit_mask():
+    L, w = 50, 9  # |i - j| <= 4
+    q, k, v = _rand_qkv(1, L, 2, 8, seed=1)
+    i = np.arange(L)
+    admit = np.abs(i[:, None] - i[None, :]) <= w // 2
+    got = oracle.attention("swa", q, k, v, 1, 1, w, centred=True)
+    np.testing.assert_allclose(got, _masked_softmax_attention(q, k, v, admit), rtol=0, atol=1e-13)
+
+
+def test_centred_half_window_zero_returns_own_value():
+    q, k, v = _rand_qkv(1, 20, 3, 4, seed=2)
+    got = oracle.attention("dswa", q, k, v, 4, 2, 1, centred=True)
+    np.testing.assert_array_equal(got, v.astype(np.float64))
+
+
+def test_centred_dswa_wide_window_is_attention_within_frame_class():
+    P, dil, L = 5, 3, 40  # frames 0..7, classes f mod 3
+    q, k, v = _rand_qkv(1, L, 2, 8, seed=3)
+    f = np.arange(L) // P
+    admit = (f[:, None] % dil) == (f[None, :] % dil)
+    got = oracle.attention("dswa", q, k, v, P, dil, 10 * L, centred=True)
+    np.testing.assert_allclose(got, _masked_softmax_attention(q, k, v, admit), rtol=0, atol=1e-13)
+
+
+def test_rope_single_pair_scores_are_cosines_of_the_position_gap():
+    # d = 2: q_t = k_t = (1, 0) and base irrelevant (theta_0 = 1), so
+    # s_ij = cos(i - j) / sqrt(2) exactly; v_t = t picks out the weights.
+    L = 12
+    q = np.zeros((1, L, 1, 2), np.float32)
+    q[..., 0] = 1.0
+    k = q.copy()
+    v = np.arange(L, dtype=np.float32).reshape(1, L, 1, 1) * np.ones((1, 1, 1, 2), np.float32)
+    got = oracle.attention("swa", q, k, v, 1, 1, 1000, centred=True, rope_base=10000.0)
+    i = np.arange(L)
+    s = np.cos(i[:, None] - i[None, :]) / math.sqrt(2.0)
+    p = np.exp(s - s.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    np.testing.assert_allclose(got[0, :, 0, 0], p @ i, rtol=0, atol=1e-12)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    # prepending tokens shifts every position by c; rows whose window does not
+    # reach the prefix must come out the same
+    c, L, w = 7, 30, 9
+    q, k, v = _rand_qkv(1, L, 2, 16, seed=4)
+    jq, jk, jv = _rand_qkv(1, c, 2, 16, seed=5)
+    cat = lambda a, b: np.concatenate([a, b], axis=1)
+    base = oracle.attention("swa", q, k, v, 1, 1, w, centred=True, rope_base=500.0)
+    shifted = oracle.attention("swa", cat(jq, q), cat(jk, k), cat(jv, v), 1, 1, w, centred=True,
+                               rope_base=500.0)[:, c:]
+    rows = slice(w // 2, L - w // 2)
+    np.testing.assert_allclose(shifted[:, rows], base[:, rows], rtol=0, atol=1e-12)
+    # and rotation is not the identity: without it the outputs differ
+    plain = oracle.attention("swa", q, k, v, 1, 1, w, centred=True)
+    assert np.abs(plain - base).max() > 1e-3
