@@ -7,7 +7,9 @@ CUDA for sm_100a behind the C ABI of ``include/hlta.h``); this package is the
 Python binding.
 """
 from .binding import (HLTA, Config, HltaError, load_library, header_symbols, LIB_PATH,
-                      BRANCH_SWA, BRANCH_DSWA, BRANCH_GDN, BRANCH_ALL, GDN_DECAYED, GDN_PAGES)
+                      BRANCH_SWA, BRANCH_DSWA, BRANCH_GDN, BRANCH_ALL, GDN_DECAYED, GDN_PAGES,
+                      WINDOW_CAUSAL, WINDOW_CENTRED)
 
 __all__ = ["HLTA", "Config", "HltaError", "load_library", "header_symbols", "LIB_PATH",
-           "BRANCH_SWA", "BRANCH_DSWA", "BRANCH_GDN", "BRANCH_ALL", "GDN_DECAYED", "GDN_PAGES"]
+           "BRANCH_SWA", "BRANCH_DSWA", "BRANCH_GDN", "BRANCH_ALL", "GDN_DECAYED", "GDN_PAGES",
+           "WINDOW_CAUSAL", "WINDOW_CENTRED"]

@@ -21,13 +21,15 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "hlta.h")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_DEVICE_TIMEOUT, ERR_INJECTED = range(7)
 BF16, FP32 = 0, 1
 GDN_DECAYED, GDN_PAGES = 0, 1
+WINDOW_CAUSAL, WINDOW_CENTRED = 0, 1
 BRANCH_SWA, BRANCH_DSWA, BRANCH_GDN, BRANCH_ALL = 1, 2, 4, 7
 
 
 class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "B", "H", "d_k", "d_v", "tokens_per_frame", "swa_window", "dswa_window",
-        "dswa_dilation", "chunk", "dtype", "max_seq_len", "max_stream_tokens", "gdn_form")]
+        "dswa_dilation", "chunk", "dtype", "max_seq_len", "max_stream_tokens", "gdn_form",
+        "window_mode")] + [("rope_base", ctypes.c_float)]
 
 
 class ProfileData(ctypes.Structure):
@@ -125,20 +127,23 @@ class HLTA:
     """One configured layer (a handle of the C library) on the current GPU."""
 
     def __init__(self, B, H, d_k, d_v, tokens_per_frame, swa_window, dswa_window, dilation,
-                 chunk=64, dtype="bf16", max_seq_len=1, max_stream_tokens=0, gdn_form=0):
+                 chunk=64, dtype="bf16", max_seq_len=1, max_stream_tokens=0, gdn_form=0,
+                 window_mode=0, rope_base=0.0):
         self.lib = load_library()
         self.cfg = Config(B, H, d_k, d_v, tokens_per_frame, swa_window, dswa_window, dilation,
                           chunk, BF16 if dtype == "bf16" else FP32, max_seq_len, max_stream_tokens,
-                          gdn_form)
+                          gdn_form, window_mode, rope_base)
         self.dtype = dtype
         h = ctypes.c_void_p()
         _check(self.lib, self.lib.hlta_create(ctypes.byref(self.cfg), ctypes.byref(h)))
         self.h = h
 
     @classmethod
-    def for_workload(cls, wl, max_seq_len=None, max_stream_tokens=0, gdn_form=0):
+    def for_workload(cls, wl, max_seq_len=None, max_stream_tokens=0, gdn_form=0, window_mode=0,
+                     rope_base=0.0):
         return cls(wl.B, wl.H, wl.d_k, wl.d_v, wl.P, wl.swa_window, wl.dswa_window, wl.dilation,
-                   wl.chunk, wl.dtype, max_seq_len or wl.L, max_stream_tokens, gdn_form)
+                   wl.chunk, wl.dtype, max_seq_len or wl.L, max_stream_tokens, gdn_form, window_mode,
+                   rope_base)
 
     def close(self):
         if getattr(self, "h", None):

@@ -1,11 +1,12 @@
 // attn_simt.cu -- CUDA-core softmax attention over the SWA / DSWA windows.
 //
-// Kairos paper, section 2.2.2: SWA (Eq. (7), causal window of w keys) and DSWA
-// (Eq. (8), SWA over residue classes of frames).  This kernel enumerates
-// exactly the keys a query admits:
+// Kairos paper, section 2.2.2: SWA (Eq. (7), causal window of w keys, or the
+// centred window as printed) and DSWA (Eq. (8), SWA over residue classes of
+// frames).  This kernel enumerates exactly the keys a query admits:
 //   f = t / P, s = t % P, class g = f % dil, m = f / dil, r = m*P + s,
-//   keys: frames f' = g + dil*m' (m' <= m) and spatial s' with
-//         r - w < m'*P + s' <= r.
+//   keys: frames f' = g + dil*m' and spatial s' with
+//         r - w < m'*P + s' <= r + w_hi   (w_hi = 0: causal)
+//   at positions below n_keys.
 // SWA is the dil = 1 case.  fp32 arithmetic throughout; it serves the fp32
 // configuration, sequences whose length is not a whole number of frames, and
 // streaming steps.  The bf16 tensor-core kernel handles full sequences.
@@ -43,7 +44,11 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnSimtArgs a) {
     const long long f_i = p_i / g.P, s_i = p_i % g.P;
     const long long grp = f_i % g.dil, m_i = f_i / g.dil;
     const long long r_i = m_i * g.P + s_i;
-    const long long r_lo = r_i - g.w + 1;
+    const long long r_lo = r_i - g.w + 1, r_hi = r_i + g.w_hi;
+    // the last class frame holding keys
+    const long long f_last = (a.n_keys - 1) / g.P;
+    const long long m_last = f_last >= grp ? (f_last - grp) / g.dil : -1;
+    const long long m_top = r_hi / g.P < m_last ? r_hi / g.P : m_last;
 
     const T *kbase = static_cast<const T *>(a.k);
     const T *vbase = static_cast<const T *>(a.v);
@@ -52,12 +57,13 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnSimtArgs a) {
 #pragma unroll
     for (int c = 0; c < OV; ++c) o[c] = 0.f;
 
-    for (long long m = m_i; m >= 0; --m) {
+    for (long long m = m_top; m >= 0; --m) {
         const long long base_r = m * g.P;
         if (base_r + g.P - 1 < r_lo) break;
         const long long s_lo = r_lo - base_r > 0 ? r_lo - base_r : 0;
-        const long long s_hi = (r_i - base_r < g.P - 1) ? r_i - base_r : g.P - 1;
         const long long p_base = (grp + (long long)g.dil * m) * g.P;
+        long long s_hi = (r_hi - base_r < g.P - 1) ? r_hi - base_r : g.P - 1;
+        if (s_hi > a.n_keys - 1 - p_base) s_hi = a.n_keys - 1 - p_base;
         for (long long s0 = s_lo; s0 <= s_hi; s0 += 32) {
             const long long s = s0 + lane;
             const bool act = s <= s_hi;

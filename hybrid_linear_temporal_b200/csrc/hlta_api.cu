@@ -91,6 +91,8 @@ struct hlta_handle {
     cudaStream_t side = nullptr;
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     float *acc2 = nullptr;
+    // rotated q and k for the attention branches (rope_base > 0)
+    void *q_rot = nullptr, *k_rot = nullptr;
     // profiling (hlta_profile_enable)
     bool prof = false;
     struct Mark {
@@ -136,6 +138,14 @@ hlta_status check_config(const hlta_config *c) {
     if (c->max_stream_tokens < 0) return fail(HLTA_ERR_INVALID_ARG, "max_stream_tokens must be >= 0");
     if (c->gdn_form != HLTA_GDN_DECAYED && c->gdn_form != HLTA_GDN_PAGES)
         return fail(HLTA_ERR_INVALID_ARG, "gdn_form must be HLTA_GDN_DECAYED or HLTA_GDN_PAGES");
+    if (c->window_mode != HLTA_WINDOW_CAUSAL && c->window_mode != HLTA_WINDOW_CENTRED)
+        return fail(HLTA_ERR_INVALID_ARG, "window_mode must be HLTA_WINDOW_CAUSAL or HLTA_WINDOW_CENTRED");
+    if (!(c->rope_base >= 0.f) || c->rope_base > 1e30f)
+        return fail(HLTA_ERR_INVALID_ARG, "rope_base must be a finite value >= 0");
+    if (c->window_mode == HLTA_WINDOW_CENTRED && c->max_stream_tokens > 0)
+        return fail(HLTA_ERR_UNSUPPORTED, "centred windows need the whole sequence: not with streaming");
+    if (c->rope_base > 0.f && c->window_mode != HLTA_WINDOW_CENTRED)
+        return fail(HLTA_ERR_UNSUPPORTED, "rotary embedding is provided with centred windows");
     if ((c->d_k != 64 && c->d_k != 128) || (c->d_v != 64 && c->d_v != 128))
         return fail(HLTA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128");
     if (c->chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64");
@@ -199,6 +209,22 @@ int out_mode(int idx, int n) {
     return idx == n - 1 ? hlta::OUT_FINAL : hlta::OUT_ADD;
 }
 
+// Window geometry of attention branch br (0 = SWA, 1 = DSWA).
+hlta::WindowGeom window_of(const hlta_config &c, int br) {
+    hlta::WindowGeom g;
+    g.P = c.tokens_per_frame;
+    g.dil = br == 0 ? 1 : c.dswa_dilation;
+    const int w = br == 0 ? c.swa_window : c.dswa_window;
+    if (c.window_mode == HLTA_WINDOW_CENTRED) {
+        g.w = w / 2 + 1;  // r - w/2 <= r_k
+        g.w_hi = w / 2;   // r_k <= r + w/2
+    } else {
+        g.w = w;
+        g.w_hi = 0;
+    }
+    return g;
+}
+
 // Run the selected branches of one pass.
 //   nq queries at absolute positions pos0 .. pos0+nq-1 (q, alpha, beta, k, v of
 //   those tokens: [B, nq, ...]); keys/values are read from (kst, vst) with
@@ -218,13 +244,28 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
         CK(cudaMemsetAsync(out, 0, (size_t)c.B * nq * c.H * c.d_v * h->elem_bytes, s));
         return HLTA_OK;
     }
-    hlta::WindowGeom geo[2];
-    geo[0].P = geo[1].P = c.tokens_per_frame;
-    geo[0].dil = 1;
-    geo[0].w = c.swa_window;
-    geo[1].dil = c.dswa_dilation;
-    geo[1].w = c.dswa_window;
+    const hlta::WindowGeom geo[2] = {window_of(c, 0), window_of(c, 1)};
     const bool want_attn[2] = {(branches & 1u) != 0, (branches & 2u) != 0};
+    // the attention branches read rotated q and k when rotary embedding is on
+    // (one-shot passes only: centred windows exclude streaming)
+    Inputs att = in;
+    if (c.rope_base > 0.f && (want_attn[0] || want_attn[1])) {
+        hlta::RopeArgs r;
+        r.q = in.q;
+        r.k = kst;
+        r.q_out = h->q_rot;
+        r.k_out = h->k_rot;
+        r.B = c.B;
+        r.n = nq;
+        r.H = c.H;
+        r.d = c.d_k;
+        r.pos0 = pos0;
+        for (int m = 0; m < 64; ++m) r.inv_freq[m] = m < c.d_k / 2 ? pow((double)c.rope_base, -2.0 * m / c.d_k) : 0.0;
+        CK(hlta::launch_rope(r, bf16, s));
+        if (h->prof) h->prof_launches += 1;
+        att.q = h->q_rot;
+        kst = h->k_rot;
+    }
     // Concurrent schedule: the memory branch (prep kernels and a sequential
     // scan on B*H SMs) runs on the side stream into its own accumulator while
     // the first attention branch runs on `s`; the last attention branch waits
@@ -260,7 +301,7 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
             ProfScope ps(h, br, s);
             bool done = false;
             const int mode = last ? (idx == 0 ? hlta::OUT_FINAL_ONLY : hlta::OUT_FINAL) : hlta::OUT_STORE;
-            cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, geo[br], in.gates, br, mode, h->acc,
+            cudaError_t e = h->tc_attn->run(att.q, kst, vst, nq, geo[br], in.gates, br, mode, h->acc,
                                             last ? h->acc2 : nullptr, out, h->dev_err, s, &done);
             if (e != cudaSuccess || !done)
                 return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
@@ -275,20 +316,17 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
         ProfScope ps(h, br, s);
         int launches = 1;
         if (br == 0 || br == 1) {
-            hlta::WindowGeom g;
-            g.P = c.tokens_per_frame;
-            g.dil = br == 0 ? 1 : c.dswa_dilation;
-            g.w = br == 0 ? c.swa_window : c.dswa_window;
+            const hlta::WindowGeom g = geo[br];
             bool done = false;
             if (one_shot && h->tc_attn) {
-                cudaError_t e = h->tc_attn->run(in.q, kst, vst, nq, g, in.gates, br, mode, h->acc,
+                cudaError_t e = h->tc_attn->run(att.q, kst, vst, nq, g, in.gates, br, mode, h->acc,
                                                 nullptr, out, h->dev_err, s, &done);
                 if (e != cudaSuccess)
                     return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
             }
             if (!done) {
                 hlta::AttnSimtArgs a;
-                a.q = in.q;
+                a.q = att.q;
                 a.k = kst;
                 a.v = vst;
                 a.q_pos0 = pos0;
@@ -298,6 +336,7 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
                 a.d_k = c.d_k;
                 a.d_v = c.d_v;
                 a.key_rows = key_rows;
+                a.n_keys = pos0 + nq;
                 a.geom = g;
                 a.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d_k);
                 a.gates = in.gates;
@@ -381,6 +420,10 @@ hlta_status hlta_create(const hlta_config *cfg, hlta_handle **out) {
     };
     const size_t acc_bytes = (size_t)cfg->B * h->acc_rows * cfg->H * cfg->d_v * sizeof(float);
     bool okk = alloc((void **)&h->acc, acc_bytes) && alloc((void **)&h->dev_err, sizeof(int));
+    if (okk && cfg->rope_base > 0.f) {
+        const size_t qk_bytes = (size_t)cfg->B * cfg->max_seq_len * cfg->H * cfg->d_k * h->elem_bytes;
+        okk = alloc(&h->q_rot, qk_bytes) && alloc(&h->k_rot, qk_bytes);
+    }
     if (okk && cfg->max_stream_tokens > 0) {
         long long cap = cfg->max_stream_tokens + max_lookback(*cfg);
         cap = (cap + 127) / 128 * 128;
@@ -432,6 +475,8 @@ hlta_status hlta_destroy(hlta_handle *h) {
     cudaFree(h->ring_v);
     cudaFree(h->stage);
     cudaFree(h->acc2);
+    cudaFree(h->q_rot);
+    cudaFree(h->k_rot);
     if (h->side) cudaStreamDestroy(h->side);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);

@@ -24,7 +24,8 @@ enum DeviceError : int { DEVERR_NONE = 0, DEVERR_TIMEOUT = 1 };
 struct WindowGeom {
     int P;          // tokens per frame
     int dil;        // dilation (1 for SWA)
-    int w;          // window in (rearranged) tokens
+    int w;          // backward reach: keys at rearranged r' with r - w < r' (w >= 1, self included)
+    int w_hi;       // forward reach: r' <= r + w_hi (0 = causal)
 };
 
 // Arguments of the SIMT attention kernel.
@@ -35,6 +36,7 @@ struct AttnSimtArgs {
     long long q_pos0;
     int nq, B, H, d_k, d_v;
     long long key_rows;
+    long long n_keys;     // keys exist at positions 0 .. n_keys-1 (bounds a forward reach)
     WindowGeom geom;
     float scale_log2;     // log2(e) / sqrt(d_k)
     const float *gates;   // [H, 3]
@@ -64,6 +66,19 @@ struct RingAppendArgs {
     long long pos0, cap;
     int n, B, H, d_k, d_v, elem_bytes;
 };
+
+// Rotary position embedding of q and k for the attention branches (a reading of
+// the RoPE the pages name for the sliding-window blocks): channel pair
+// (2m, 2m+1) of the token at absolute position pos0 + t is rotated by the angle
+// (pos0 + t) * inv_freq[m], inv_freq[m] = base^(-2m/d).  Writes rotated copies.
+struct RopeArgs {
+    const void *q, *k;  // [B, n, H, d] dtype
+    void *q_out, *k_out;
+    int B, n, H, d;
+    long long pos0;
+    double inv_freq[64];
+};
+cudaError_t launch_rope(const RopeArgs &a, bool bf16, cudaStream_t s);
 
 // Sets the thread-local message returned by hlta_last_error() (empty clears it).
 void set_last_error(const char *msg);

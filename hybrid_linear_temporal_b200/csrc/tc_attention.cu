@@ -8,7 +8,8 @@
 // SWA (Pseg = L), one latent frame for DSWA (Pseg = P).  Segment f of a batch
 // belongs to class g = f mod dil at class position m = f / dil; a token s of it
 // sits at rearranged position r = m*Pseg + s, and query r attends to the keys of
-// its class with r - w < r_k <= r.  SWA is dil = 1 with one segment.  No
+// its class with r - w < r_k <= r + w_hi (w_hi = 0: the causal window; w_hi > 0:
+// the centred window Eq. (7) prints).  SWA is dil = 1 with one segment.  No
 // rearranged copy is made: TMA reads tiles straight from the caller's
 // [B, L, H, d] tensors through a 4-D view (d, H, Pseg, B*F), whose
 // out-of-range rows arrive as zeros.
@@ -69,7 +70,7 @@ struct KeyTile {
 };
 
 struct TcAttnParams {
-    int Pseg, Fseg, dil, w, qblocks_per_seg;
+    int Pseg, Fseg, dil, w, w_hi, qblocks_per_seg;
     int H, L;
     float scale_log2;
     const float *gates;
@@ -169,12 +170,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         int n = 0;
-        const int lo_r = r_min - p.w + 1;
+        const int lo_r = r_min - p.w + 1, hi_r = r_max + p.w_hi;
         const int nqs[kQT] = {nq0, nq1};
-        for (int mm = m; mm >= 0; --mm) {
+        // class positions from the last one the forward reach touches down to the
+        // first the backward reach touches
+        const int m_last = (p.Fseg - 1 - g) / p.dil;
+        for (int mm = min(m_last, hi_r / p.Pseg); mm >= 0; --mm) {
             const int base = mm * p.Pseg;
             if (base + p.Pseg - 1 < lo_r) break;
-            const int s_lo = max(0, lo_r - base), s_hi = min(p.Pseg - 1, r_max - base);
+            const int s_lo = max(0, lo_r - base), s_hi = min(p.Pseg - 1, hi_r - base);
             for (int t = s_lo / kBN; t <= s_hi / kBN && n < kMaxKT; ++t, ++n) {
                 KeyTile &k = sm.kt[n];
                 k.seg = b * p.Fseg + g + p.dil * mm;
@@ -184,8 +188,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                 for (int j = 0; j < kQT; ++j) {
                     const int lo = r_min + j * kBM, hi = lo + nqs[j] - 1;
-                    k.use[j] = nqs[j] > 0 && k.rbase <= hi && k.rbase + k.kvalid - 1 >= lo - p.w + 1;
-                    k.full[j] = k.kvalid == kBN && k.rbase + kBN - 1 <= lo && k.rbase > hi - p.w;
+                    k.use[j] = nqs[j] > 0 && k.rbase <= hi + p.w_hi && k.rbase + k.kvalid - 1 >= lo - p.w + 1;
+                    k.full[j] = k.kvalid == kBN && k.rbase + kBN - 1 <= lo + p.w_hi && k.rbase > hi - p.w;
                 }
             }
         }
@@ -352,7 +356,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tmem_wait_ld();
             if (!full) {
                 const int lo = max(0, r_q - p.w + 1 - rbase);
-                const int hi = min(kvalid - 1, r_q - rbase);
+                const int hi = min(kvalid - 1, r_q + p.w_hi - rbase);
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
@@ -486,7 +490,7 @@ public:
         if (*Pseg < kBN) return false;
         // key tiles one CTA can need: the span w + 2*kBM - 1 rearranged rows, cut
         // at most at every segment boundary it crosses
-        const long long span = (long long)g.w + kQT * kBM - 1;
+        const long long span = (long long)g.w + g.w_hi + kQT * kBM - 1;
         const long long bound = (span + kBN - 1) / kBN + 2 * (span / *Pseg + 2);
         if (bound > kMaxKT) return false;
         return (long long)*Fseg * *Pseg <= (1LL << 30);
@@ -514,6 +518,7 @@ public:
         p.Fseg = Fseg;
         p.dil = g.dil;
         p.w = g.w;
+        p.w_hi = g.w_hi;
         p.qblocks_per_seg = (Pseg + kQT * kBM - 1) / (kQT * kBM);
         p.H = cfg_.H;
         p.L = L;

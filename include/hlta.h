@@ -85,6 +85,14 @@ enum {
  *                     a unit k_t. */
 enum { HLTA_GDN_DECAYED = 0, HLTA_GDN_PAGES = 1 };
 
+/* Attention window (hlta_config.window_mode), in (rearranged, for DSWA) token
+ * positions r, with w the branch's window:
+ *   HLTA_WINDOW_CAUSAL   keys r - w < r_k <= r: the w most recent keys (default).
+ *   HLTA_WINDOW_CENTRED  keys |r_k - r| <= floor(w/2): the centred window Eq. (7)
+ *                        prints, for in-clip (bidirectional) use.  One-shot
+ *                        hlta_forward only: not with streaming. */
+enum { HLTA_WINDOW_CAUSAL = 0, HLTA_WINDOW_CENTRED = 1 };
+
 /* Layer configuration, fixed for the life of a handle. */
 typedef struct {
     int B;                 /* batch, >= 1 */
@@ -100,6 +108,11 @@ typedef struct {
     int max_seq_len;       /* largest L accepted by hlta_forward (>= 1) */
     int max_stream_tokens; /* largest n of hlta_stream_step; 0 disables streaming */
     int gdn_form;          /* HLTA_GDN_DECAYED (0) or HLTA_GDN_PAGES (1) */
+    int window_mode;       /* HLTA_WINDOW_CAUSAL (0) or HLTA_WINDOW_CENTRED (1) */
+    float rope_base;       /* > 0: rotary embedding of q and k for SWA/DSWA (the pages name
+                              RoPE for these blocks; reading: channel pair (2m, 2m+1) of the
+                              token at position t turns by t * rope_base^(-2m/d_k)); 0: none.
+                              Centred windows only.  The memory branch never rotates. */
 } hlta_config;
 
 typedef struct hlta_handle hlta_handle;

@@ -60,19 +60,23 @@ def sample_rows(wl, n: int, seed: int = 0) -> np.ndarray:
     return np.unique(np.array(rows, dtype=np.int64))
 
 
-def oracle_rows(inp: Inputs, rows, gdn_out=None, branches=("swa", "dswa", "gdn")):
+def oracle_rows(inp: Inputs, rows, gdn_out=None, branches=("swa", "dswa", "gdn"), centred=False,
+                rope_base=0.0):
     """Oracle layer output at the given rows ([n, d_v] float64).  gdn_out: a full
-    oracle GDN output [B,L,H,d_v] (computed when None and GDN is selected)."""
+    oracle GDN output [B,L,H,d_v] (computed when None and GDN is selected).
+    centred / rope_base select the centred attention window and the rotary
+    embedding of the attention branches."""
     wl = inp.wl
     g = inp.gates.astype(np.float64)
     h = rows % wl.H
     res = np.zeros((rows.size, wl.d_v))
+    kw = dict(centred=centred, rope_base=rope_base)
     if "swa" in branches:
         res += g[h, 0, None] * oracle.attention_rows("swa", inp.q, inp.k, inp.v, wl.P, 1,
-                                                     wl.swa_window, rows)
+                                                     wl.swa_window, rows, **kw)
     if "dswa" in branches:
         res += g[h, 1, None] * oracle.attention_rows("dswa", inp.q, inp.k, inp.v, wl.P,
-                                                     wl.dilation, wl.dswa_window, rows)
+                                                     wl.dilation, wl.dswa_window, rows, **kw)
     if "gdn" in branches:
         if gdn_out is None:
             gdn_out, _ = oracle.gdn(inp.q, inp.k, inp.v, inp.alpha, inp.beta)

@@ -38,7 +38,7 @@ def test_version(lib):
 def _cfg(**kw):
     base = dict(B=1, H=2, d_k=64, d_v=64, tokens_per_frame=4, swa_window=8, dswa_window=8,
                 dswa_dilation=2, chunk=64, dtype=binding.BF16, max_seq_len=128, max_stream_tokens=0,
-                gdn_form=binding.GDN_DECAYED)
+                gdn_form=binding.GDN_DECAYED, window_mode=binding.WINDOW_CAUSAL, rope_base=0.0)
     base.update(kw)
     return binding.Config(*[base[n] for n, _ in binding.Config._fields_])
 
@@ -54,6 +54,25 @@ def _cfg(**kw):
 def test_create_rejects_bad_config_before_device(lib, field, value, status):
     h = ctypes.c_void_p()
     st = lib.hlta_create(ctypes.byref(_cfg(**{field: value})), ctypes.byref(h))
+    assert st == status
+    assert h.value is None
+    assert lib.hlta_last_error().decode()
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(window_mode=2), binding.ERR_INVALID_ARG),
+    (dict(window_mode=-1), binding.ERR_INVALID_ARG),
+    (dict(window_mode=binding.WINDOW_CENTRED, rope_base=-1.0), binding.ERR_INVALID_ARG),
+    (dict(window_mode=binding.WINDOW_CENTRED, rope_base=float("nan")), binding.ERR_INVALID_ARG),
+    (dict(window_mode=binding.WINDOW_CENTRED, rope_base=float("inf")), binding.ERR_INVALID_ARG),
+    # the rotary embedding is offered with the centred (in-clip) window only
+    (dict(window_mode=binding.WINDOW_CAUSAL, rope_base=10000.0), binding.ERR_UNSUPPORTED),
+    # a centred window reaches keys after the query: not available token by token
+    (dict(window_mode=binding.WINDOW_CENTRED, max_stream_tokens=16), binding.ERR_UNSUPPORTED),
+])
+def test_create_rejects_bad_window_config(lib, over, status):
+    h = ctypes.c_void_p()
+    st = lib.hlta_create(ctypes.byref(_cfg(**over)), ctypes.byref(h))
     assert st == status
     assert h.value is None
     assert lib.hlta_last_error().decode()

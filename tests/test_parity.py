@@ -105,6 +105,88 @@ def test_initial_state_and_stress_inputs(torch_cuda):
     full_compare(torch_cuda, wl, seed=2, q_scale=384.0, branches=("swa", "dswa"))
 
 
+BRANCHES = ("swa", "dswa", "gdn")
+
+
+def centred_compare(torch_cuda, wl, rope_base, seed=0, q_scale=1.0, branches=BRANCHES):
+    """The centred window (Eq. (7) as printed, and DSWA over it) with or without
+    the rotary embedding of q and k, against the oracle: the layer and each
+    selected attention branch on every element."""
+    from hybrid_linear_temporal_b200 import WINDOW_CENTRED
+    inp = make_inputs(wl, seed=seed, q_scale=q_scale)
+    g = inp.gates.astype(np.float64)
+    ref = {}
+    for name, dil, w in (("swa", 1, wl.swa_window), ("dswa", wl.dilation, wl.dswa_window)):
+        if name in branches:
+            ref[name] = oracle.attention(name, inp.q, inp.k, inp.v, wl.P, dil, w, centred=True,
+                                         rope_base=rope_base)
+    if "gdn" in branches:
+        ref["gdn"], _ = oracle.gdn(inp.q, inp.k, inp.v, inp.alpha, inp.beta)
+    total = sum(g[None, None, :, i, None] * ref[n] for i, n in enumerate(BRANCHES) if n in branches)
+    layer = layer_for(wl, window_mode=WINDOW_CENTRED, rope_base=rope_base)
+    dev = to_device(inp)
+    mask = sum(1 << i for i, n in enumerate(BRANCHES) if n in branches)
+    out, _ = run_gpu(layer, dev, branches=mask)
+    assert_close(to_numpy64(out), total, wl.dtype, f"{wl.name} centred layer")
+    got = {}
+    for i, name in enumerate(BRANCHES[:2]):
+        if name in branches:
+            o, _ = run_gpu(layer, dev, branches=1 << i)
+            got[name] = to_numpy64(o)
+            assert_close(got[name], g[None, None, :, i, None] * ref[name], wl.dtype,
+                         f"{wl.name} centred branch {name}")
+    layer.close()
+    return inp, got
+
+
+# Scaled queries sharpen the softmax so that the rotation shows in the result;
+# they also scale the memory branch's output, so those cases compare the
+# attention branches alone (the memory branch never sees the rotation).
+@pytest.mark.parametrize("rope_base,q_scale,branches", [
+    (0.0, 1.0, BRANCHES), (10000.0, 1.0, BRANCHES), (10000.0, 16.0, BRANCHES[:2])])
+def test_centred_tiny_fp32(torch_cuda, rope_base, q_scale, branches):
+    """CUDA-core attention over the centred window (P = 1: DSWA dilates tokens)."""
+    centred_compare(torch_cuda, WORKLOADS["tiny_fp32"], rope_base, q_scale=q_scale, branches=branches)
+
+
+@pytest.mark.parametrize("rope_base,q_scale,branches", [
+    (0.0, 1.0, BRANCHES), (10000.0, 1.0, BRANCHES), (10000.0, 16.0, BRANCHES[:2]),
+    (500.0, 64.0, BRANCHES[:2])])
+def test_centred_clip_4k_bf16(torch_cuda, rope_base, q_scale, branches):
+    """Tensor-core attention over the centred window, with and without rotation."""
+    wl = WORKLOADS["clip_4k"]
+    inp, got = centred_compare(torch_cuda, wl, rope_base, q_scale=q_scale, branches=branches)
+    if rope_base > 0 and q_scale > 1:
+        # the rotation is visible: the unrotated oracle is far from the result
+        g = inp.gates.astype(np.float64)[None, None, :, 0, None]
+        plain = oracle.attention("swa", inp.q, inp.k, inp.v, wl.P, 1, wl.swa_window, centred=True)
+        assert errors(got["swa"], g * plain)["rel_l2"] > 10 * 5e-3
+
+
+@pytest.mark.parametrize("case", [
+    dict(L=1), dict(L=65), dict(L=333, P=50), dict(L=256, swa_window=1, dswa_window=1),
+    dict(L=256, swa_window=2, dswa_window=3), dict(L=300, swa_window=1000, dswa_window=1000),
+    dict(L=384, P=8, dilation=5, dswa_window=41), dict(L=512, d_k=64, d_v=64),
+    dict(B=2, L=640, H=3, P=128, swa_window=301),
+])
+def test_centred_edge_cases_bf16(torch_cuda, case):
+    base = WORKLOADS["clip_4k"].with_(H=2, L=256, P=32, swa_window=48, dswa_window=40, dilation=3)
+    centred_compare(torch_cuda, base.with_(**case), 10000.0, q_scale=16.0, branches=BRANCHES[:2])
+
+
+def test_centred_rollout_480p_sampled(torch_cuda):
+    """The 480P-shaped rollout with the centred window and rotation: sampled rows."""
+    from hybrid_linear_temporal_b200 import WINDOW_CENTRED
+    wl = WORKLOADS["rollout_480p"]
+    inp = make_inputs(wl, q_scale=16.0)
+    layer = layer_for(wl, window_mode=WINDOW_CENTRED, rope_base=10000.0)
+    out, _ = run_gpu(layer, to_device(inp), branches=3)
+    rows = sample_rows(wl, 2000)
+    ref = oracle_rows(inp, rows, branches=("swa", "dswa"), centred=True, rope_base=10000.0)
+    assert_close(to_numpy64(out).reshape(-1, wl.d_v)[rows], ref, wl.dtype, "rollout centred rows")
+    layer.close()
+
+
 def _sampled_compare(torch_cuda, wl, n_rows, heads_for_state=None):
     inp = make_inputs(wl)
     layer = layer_for(wl)
