@@ -1,4 +1,5 @@
-"""fp64 CPU oracle of the Hybrid Linear Temporal Attention forward pass.
+"""fp64 CPU oracle of the Hybrid Linear Temporal Attention layer (forward pass
+and its reverse-mode derivatives).
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, the package smoke check and
 the benchmark's CPU-baseline leg, never by the product path.  It shares no
@@ -16,7 +17,7 @@ Two independent implementations:
 Parity pins of every function: ``tests/test_oracle.py``.
 """
 from .core import (attention, attention_rows, forward, gdn, gdn_chunked, num_threads,
-                   build, library_path, dswa_span)
+                   build, library_path, dswa_span, attention_backward, gdn_backward, backward)
 
 __all__ = ["attention", "attention_rows", "forward", "gdn", "gdn_chunked", "num_threads",
-           "build", "library_path", "dswa_span"]
+           "build", "library_path", "dswa_span", "attention_backward", "gdn_backward", "backward"]

@@ -46,6 +46,12 @@ def _load():
         lib.oracle_gdn.restype = i
         lib.oracle_gdn_chunked.argtypes = [i, i, i, i, i, vp, vp, vp, i, fp, fp, dp, dp, dp, i]
         lib.oracle_gdn_chunked.restype = i
+        lib.oracle_attention_backward.argtypes = [i, i, ctypes.c_double, i, i, i, i, i, i, i, i,
+                                                  vp, vp, vp, i, dp, dp, dp, dp]
+        lib.oracle_attention_backward.restype = i
+        lib.oracle_gdn_backward.argtypes = [i, i, i, i, i, vp, vp, vp, i, fp, fp, dp, dp, dp, dp, dp,
+                                            dp, dp, dp, dp, i]
+        lib.oracle_gdn_backward.restype = i
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i
         _lib = lib
@@ -198,4 +204,89 @@ def forward(inp, S0=None, branches=("swa", "dswa", "gdn"), variant=0):
         res["gdn"] = o
         total = total + g[None, None, :, 2, None] * o
     res["out"] = total
+    return res
+
+
+def attention_backward(kind: str, q, k, v, P: int, dilation: int, w: int, dO, centred: bool = False,
+                       rope_base: float = 0.0):
+    """Derivatives (dq, dk, dv) of ``attention`` given dO = dLoss/dO [B,L,H,d_v]
+    (oracle_attention_backward in hlta_oracle.c).  float64 arrays."""
+    lib = _load()
+    q, dt = _tensor(q)
+    k, _ = _tensor(k)
+    v, _ = _tensor(v)
+    B, L, H, dk_ = q.shape
+    dv_ = v.shape[-1]
+    dO = np.ascontiguousarray(dO, dtype=np.float64)
+    assert dO.shape == (B, L, H, dv_)
+    dq = np.empty((B, L, H, dk_))
+    dk = np.empty((B, L, H, dk_))
+    dv = np.empty((B, L, H, dv_))
+    rc = lib.oracle_attention_backward({"swa": 0, "dswa": 1}[kind], int(centred), float(rope_base),
+                                       B, L, H, dk_, dv_, P, dilation, w, q.ctypes.data, k.ctypes.data,
+                                       v.ctypes.data, dt, _dptr(dO), _dptr(dq), _dptr(dk), _dptr(dv))
+    if rc != 0:
+        raise ValueError("oracle_attention_backward: bad arguments")
+    return dq, dk, dv
+
+
+def gdn_backward(q, k, v, alpha, beta, dO, S0=None, dS_final=None, variant: int = 0):
+    """Derivatives of ``gdn`` given dO [B,L,H,d_v] and the gradient of the final
+    state dS_final [B,H,d_v,d_k] (None: zero).  Returns a dict of float64 arrays
+    dq, dk, dv, dalpha, dbeta, dS0 (oracle_gdn_backward in hlta_oracle.c)."""
+    lib = _load()
+    q, k, v, dt, ap, bp, S0, (B, L, H, dk_, dv_) = _gdn_common(q, k, v, alpha, beta, S0)
+    dO = np.ascontiguousarray(dO, dtype=np.float64)
+    assert dO.shape == (B, L, H, dv_)
+    if dS_final is not None:
+        dS_final = np.ascontiguousarray(dS_final, dtype=np.float64)
+        assert dS_final.shape == (B, H, dv_, dk_)
+    r = {"dq": np.empty((B, L, H, dk_)), "dk": np.empty((B, L, H, dk_)), "dv": np.empty((B, L, H, dv_)),
+         "dalpha": np.empty((B, L, H)), "dbeta": np.empty((B, L, H)), "dS0": np.empty((B, H, dv_, dk_))}
+    rc = lib.oracle_gdn_backward(B, L, H, dk_, dv_, q.ctypes.data, k.ctypes.data, v.ctypes.data, dt, ap,
+                                 bp, _dptr(S0), _dptr(dO), _dptr(dS_final), _dptr(r["dq"]),
+                                 _dptr(r["dk"]), _dptr(r["dv"]), _dptr(r["dalpha"]), _dptr(r["dbeta"]),
+                                 _dptr(r["dS0"]), variant)
+    if rc != 0:
+        raise ValueError("oracle_gdn_backward: bad arguments")
+    return r
+
+
+def backward(inp, dout, S0=None, dS_final=None, branches=("swa", "dswa", "gdn"), variant=0,
+             centred=False, rope_base=0.0):
+    """Derivatives of the whole layer out = sum_b g[h, b] O_b given dout =
+    dLoss/dout [B,L,H,d_v] and dS_final (gradient of the final memory state).
+
+    Each branch receives dO_b = g[h, b] dout; dgates[h, b] = sum over batch,
+    tokens and channels of dout * O_b.  Returns a dict of float64 arrays: dq,
+    dk, dv, dalpha, dbeta (zero when the memory branch is not selected), dgates
+    [H, 3] and dS0 (None when the memory branch is not selected).
+    """
+    wl = inp.wl
+    dout = np.asarray(dout, dtype=np.float64)
+    g = inp.gates.astype(np.float64)
+    B, L, H = wl.B, wl.L, wl.H
+    res = {"dq": np.zeros((B, L, H, wl.d_k)), "dk": np.zeros((B, L, H, wl.d_k)),
+           "dv": np.zeros((B, L, H, wl.d_v)), "dalpha": np.zeros((B, L, H)),
+           "dbeta": np.zeros((B, L, H)), "dgates": np.zeros((H, 3)), "dS0": None}
+    kw = dict(centred=centred, rope_base=rope_base)
+    for col, (name, dil, w) in enumerate((("swa", 1, wl.swa_window),
+                                          ("dswa", wl.dilation, wl.dswa_window))):
+        if name not in branches:
+            continue
+        o = attention(name, inp.q, inp.k, inp.v, wl.P, dil, w, **kw)
+        res["dgates"][:, col] = np.einsum("blhc,blhc->h", dout, o)
+        dq, dk, dv = attention_backward(name, inp.q, inp.k, inp.v, wl.P, dil, w,
+                                        g[None, None, :, col, None] * dout, **kw)
+        res["dq"] += dq
+        res["dk"] += dk
+        res["dv"] += dv
+    if "gdn" in branches:
+        o, _ = gdn(inp.q, inp.k, inp.v, inp.alpha, inp.beta, S0, variant=variant)
+        res["dgates"][:, 2] = np.einsum("blhc,blhc->h", dout, o)
+        r = gdn_backward(inp.q, inp.k, inp.v, inp.alpha, inp.beta, g[None, None, :, 2, None] * dout,
+                         S0, dS_final, variant)
+        for n in ("dq", "dk", "dv", "dalpha", "dbeta"):
+            res[n] += r[n]
+        res["dS0"] = r["dS0"]
     return res

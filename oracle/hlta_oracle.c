@@ -28,6 +28,9 @@
  *   oracle_gdn_chunked-- the same recurrence regrouped into chunks (a
  *                        derivation from Eq. (6), not on the pages); used only to
  *                        show that the chunk form computes the recurrence.
+ *   oracle_attention_backward, oracle_gdn_backward -- reverse-mode derivatives
+ *                        of the two forward definitions (the chain rule applied
+ *                        to them step by step; the pages print no backward).
  *
  * Parity pins for every function live in tests/test_oracle.py.
  */
@@ -428,4 +431,300 @@ int oracle_num_threads(void) {
 #else
     return 1;
 #endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass (reverse-mode derivatives of the functions above).         */
+/* The pages train the layer but print no backward formulas; the ones below */
+/* are the chain rule applied to the forward definitions, step by step.     */
+/* ------------------------------------------------------------------------ */
+
+/* Transpose of rope_rotate: maps the gradient of the rotated vector to the
+ * gradient of the unrotated one (rotation by -theta). */
+static void rope_unrotate(double *g, int d, long t, double base) {
+    for (int m = 0; 2 * m + 1 < d; ++m) {
+        double theta = (double)t * pow(base, -2.0 * m / (double)d);
+        double c = cos(theta), sn = sin(theta);
+        double a = g[2 * m], b = g[2 * m + 1];
+        g[2 * m] = a * c + b * sn;
+        g[2 * m + 1] = -a * sn + b * c;
+    }
+}
+
+/*
+ * oracle_attention_backward: derivatives of the attention rows of
+ * attention_core (same kind / centred / rope_base / window arguments) with
+ * respect to q, k and v, given dO = dLoss/dO for every row [B,L,H,d_v].
+ * For query i with admitted keys J(i), logits s_j = q_i.k_j / sqrt(d_k) and
+ * p = softmax(s):
+ *   dv_j += p_j dO_i
+ *   dp_j  = dO_i . v_j,   ds_j = p_j (dp_j - sum_m p_m dp_m)
+ *   dq_i += sum_j ds_j k_j / sqrt(d_k),   dk_j += ds_j q_i / sqrt(d_k)
+ * With rotary embedding q, k above are the rotated vectors and the results are
+ * mapped back through the transposed rotation.
+ * dq, dk: [B,L,H,d_k], dv: [B,L,H,d_v] doubles, overwritten.  Every key is
+ * examined (no span bound).  Returns 0, or -1 on bad arguments.
+ */
+int oracle_attention_backward(int kind, int centred, double rope_base, int B, int L, int H, int d_k,
+                              int d_v, int P, int dil, int w, const void *q, const void *k,
+                              const void *v, int dt, const double *dO, double *dq, double *dk,
+                              double *dv) {
+    if (B <= 0 || L <= 0 || H <= 0 || d_k <= 0 || d_v <= 0 || P <= 0 || dil <= 0 || w <= 0)
+        return -1;
+    if (kind != 0 && kind != 1) return -1;
+    if (rope_base < 0.0 || (rope_base > 0.0 && (d_k % 2 != 0 || !centred))) return -1;
+    const double scale = 1.0 / sqrt((double)d_k);
+    memset(dq, 0, sizeof(double) * (size_t)B * L * H * d_k);
+    memset(dk, 0, sizeof(double) * (size_t)B * L * H * d_k);
+    memset(dv, 0, sizeof(double) * (size_t)B * L * H * d_v);
+
+    /* keys accumulate over queries, so one thread owns one (b, h) */
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            double *Qr = (double *)malloc(sizeof(double) * (size_t)L * d_k);
+            double *Kr = (double *)malloc(sizeof(double) * (size_t)L * d_k);
+            double *dQr = (double *)calloc((size_t)L * d_k, sizeof(double));
+            double *dKr = (double *)calloc((size_t)L * d_k, sizeof(double));
+            double *p = (double *)malloc(sizeof(double) * (size_t)L);
+            double *dp = (double *)malloc(sizeof(double) * (size_t)L);
+            for (long t = 0; t < L; ++t) {
+                size_t off = (((size_t)b * L + t) * H + h) * d_k;
+                for (int c = 0; c < d_k; ++c) {
+                    Qr[(size_t)t * d_k + c] = load_elem(q, dt, off + c);
+                    Kr[(size_t)t * d_k + c] = load_elem(k, dt, off + c);
+                }
+                if (rope_base > 0.0) {
+                    rope_rotate(Qr + (size_t)t * d_k, d_k, t, rope_base);
+                    rope_rotate(Kr + (size_t)t * d_k, d_k, t, rope_base);
+                }
+            }
+            for (long i = 0; i < L; ++i) {
+                const double *qi = Qr + (size_t)i * d_k;
+                const double *dOi = dO + (((size_t)b * L + i) * H + h) * d_v;
+                double m = -INFINITY;
+                for (long j = 0; j < L; ++j) {
+                    int in;
+                    if (centred)
+                        in = kind == 0 ? swa_in_centred(i, j, w) : dswa_in_centred(i, j, P, dil, w);
+                    else
+                        in = kind == 0 ? swa_in_window(i, j, w) : dswa_in_window(i, j, P, dil, w);
+                    if (!in) {
+                        p[j] = NAN;
+                        continue;
+                    }
+                    double s = 0.0;
+                    for (int c = 0; c < d_k; ++c) s += qi[c] * Kr[(size_t)j * d_k + c];
+                    p[j] = s * scale;
+                    if (p[j] > m) m = p[j];
+                }
+                double denom = 0.0;
+                for (long j = 0; j < L; ++j)
+                    if (!isnan(p[j])) {
+                        p[j] = exp(p[j] - m);
+                        denom += p[j];
+                    }
+                double pdp = 0.0;
+                for (long j = 0; j < L; ++j) {
+                    if (isnan(p[j])) continue;
+                    p[j] /= denom;
+                    size_t voff = (((size_t)b * L + j) * H + h) * d_v;
+                    double s = 0.0;
+                    for (int c = 0; c < d_v; ++c) s += dOi[c] * load_elem(v, dt, voff + c);
+                    dp[j] = s;
+                    pdp += p[j] * s;
+                }
+                for (long j = 0; j < L; ++j) {
+                    if (isnan(p[j])) continue;
+                    double ds = p[j] * (dp[j] - pdp) * scale;
+                    for (int c = 0; c < d_k; ++c) {
+                        dQr[(size_t)i * d_k + c] += ds * Kr[(size_t)j * d_k + c];
+                        dKr[(size_t)j * d_k + c] += ds * qi[c];
+                    }
+                    double *dvj = dv + (((size_t)b * L + j) * H + h) * d_v;
+                    for (int c = 0; c < d_v; ++c) dvj[c] += p[j] * dOi[c];
+                }
+            }
+            for (long t = 0; t < L; ++t) {
+                if (rope_base > 0.0) {
+                    rope_unrotate(dQr + (size_t)t * d_k, d_k, t, rope_base);
+                    rope_unrotate(dKr + (size_t)t * d_k, d_k, t, rope_base);
+                }
+                size_t off = (((size_t)b * L + t) * H + h) * d_k;
+                memcpy(dq + off, dQr + (size_t)t * d_k, sizeof(double) * d_k);
+                memcpy(dk + off, dKr + (size_t)t * d_k, sizeof(double) * d_k);
+            }
+            free(Qr);
+            free(Kr);
+            free(dQr);
+            free(dKr);
+            free(p);
+            free(dp);
+        }
+    }
+    return 0;
+}
+
+/* One step of the recurrence in the form oracle_gdn_backward uses:
+ * Sn = alpha Sp + u k^T, u = beta (v - rho Sp k), rho = alpha (variant 0) or 1. */
+static void gdn_step(const double *Sp, double *Sn, const double *kt, const double *vt, double a,
+                     double be, int variant, int d_k, int d_v) {
+    const double rho = variant == 0 ? a : 1.0;
+    for (int e = 0; e < d_v; ++e) {
+        double s = 0.0;
+        for (int c = 0; c < d_k; ++c) s += Sp[(size_t)e * d_k + c] * kt[c];
+        const double u = be * (vt[e] - rho * s);
+        for (int c = 0; c < d_k; ++c) Sn[(size_t)e * d_k + c] = a * Sp[(size_t)e * d_k + c] + u * kt[c];
+    }
+}
+
+/*
+ * oracle_gdn_backward: derivatives of oracle_gdn (variant 0 or 1) with respect
+ * to q, k, v, alpha, beta and the initial state, given dO [B,L,H,d_v] and
+ * dS_final [B,H,d_v,d_k] (NULL: zero), the gradient of the final state.
+ *
+ * Both variants write the update as S_t = alpha_t S_{t-1} + u_t k_t^T with the
+ * retrieval r_t = S_{t-1} k_t and u_t = beta_t (v_t - rho_t r_t), rho_t = alpha_t
+ * (variant 0) or 1 (variant 1).  Walking t = L-1 .. 0 with G the gradient of
+ * S_t (G starts at dS_final):
+ *   G    += dO_t q_t^T;          dq_t = S_t^T dO_t
+ *   du    = G k_t;               dv_t = beta_t du;   dbeta_t = du . (v_t - rho_t r_t)
+ *   dr    = -beta_t rho_t du;    dalpha_t = <G, S_{t-1}> (+ -beta_t du . r_t, variant 0)
+ *   dk_t  = G^T u_t + S_{t-1}^T dr
+ *   G    <- alpha_t G + dr k_t^T  (the gradient of S_{t-1})
+ * and dS0 = G at the end.  S_{t-1} is needed in reverse order: the states at
+ * every 64th step are kept from a first forward sweep, and the states inside
+ * one such segment are recomputed from its first state by the same recurrence.
+ * Outputs (doubles, overwritten): dq, dk [B,L,H,d_k], dv [B,L,H,d_v], dalpha,
+ * dbeta [B,L,H], dS0 [B,H,d_v,d_k] or NULL.  Returns 0, or -1 on bad arguments.
+ */
+int oracle_gdn_backward(int B, int L, int H, int d_k, int d_v, const void *q, const void *k,
+                        const void *v, int dt, const float *alpha, const float *beta,
+                        const double *S0, const double *dO, const double *dS_final, double *dq,
+                        double *dk, double *dv, double *dalpha, double *dbeta, double *dS0,
+                        int variant) {
+    if (B <= 0 || L < 0 || H <= 0 || d_k <= 0 || d_v <= 0) return -1;
+    if (variant != 0 && variant != 1) return -1;
+    const int SEG = 64;
+    const int nseg = (L + SEG - 1) / SEG;
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            const size_t sd = (size_t)d_v * d_k;
+            /* ckpt[g]: state before segment g; seg[i]: state after step g*SEG + i */
+            double *ckpt = (double *)malloc(sizeof(double) * sd * (size_t)(nseg > 0 ? nseg : 1));
+            double *seg = (double *)malloc(sizeof(double) * sd * (size_t)(SEG + 1));
+            double *G = (double *)malloc(sizeof(double) * sd);
+            double *kt = (double *)malloc(sizeof(double) * d_k);
+            double *qt = (double *)malloc(sizeof(double) * d_k);
+            double *vt = (double *)malloc(sizeof(double) * d_v);
+            double *r = (double *)malloc(sizeof(double) * d_v);
+            double *u = (double *)malloc(sizeof(double) * d_v);
+            double *du = (double *)malloc(sizeof(double) * d_v);
+            double *dr = (double *)malloc(sizeof(double) * d_v);
+
+#define LOAD_TOKEN(t)                                                              \
+    do {                                                                           \
+        size_t row_ = ((size_t)b * L + (t)) * H + h;                               \
+        for (int c = 0; c < d_k; ++c) {                                            \
+            kt[c] = load_elem(k, dt, row_ * d_k + c);                              \
+            qt[c] = load_elem(q, dt, row_ * d_k + c);                              \
+        }                                                                          \
+        for (int c = 0; c < d_v; ++c) vt[c] = load_elem(v, dt, row_ * d_v + c);    \
+    } while (0)
+            /* forward sweep: checkpoints */
+            double *S = seg; /* scratch state */
+            if (S0)
+                memcpy(S, S0 + ((size_t)b * H + h) * sd, sizeof(double) * sd);
+            else
+                memset(S, 0, sizeof(double) * sd);
+            for (int t = 0; t < L; ++t) {
+                if (t % SEG == 0) memcpy(ckpt + (size_t)(t / SEG) * sd, S, sizeof(double) * sd);
+                size_t row = ((size_t)b * L + t) * H + h;
+                LOAD_TOKEN(t);
+                double *Sn = seg + sd;
+                gdn_step(S, Sn, kt, vt, (double)alpha[row], (double)beta[row], variant, d_k, d_v);
+                memcpy(S, Sn, sizeof(double) * sd);
+            }
+            if (dS_final)
+                memcpy(G, dS_final + ((size_t)b * H + h) * sd, sizeof(double) * sd);
+            else
+                memset(G, 0, sizeof(double) * sd);
+
+            for (int g = nseg - 1; g >= 0; --g) {
+                int t0 = g * SEG, n = (L - t0 < SEG) ? L - t0 : SEG;
+                /* recompute the segment's states: seg[0] = before, seg[i+1] = after step t0+i */
+                memcpy(seg, ckpt + (size_t)g * sd, sizeof(double) * sd);
+                for (int i = 0; i < n; ++i) {
+                    size_t row = ((size_t)b * L + t0 + i) * H + h;
+                    LOAD_TOKEN(t0 + i);
+                    gdn_step(seg + (size_t)i * sd, seg + (size_t)(i + 1) * sd, kt, vt, (double)alpha[row],
+                             (double)beta[row], variant, d_k, d_v);
+                }
+                for (int i = n - 1; i >= 0; --i) {
+                    int t = t0 + i;
+                    size_t row = ((size_t)b * L + t) * H + h;
+                    const double a = (double)alpha[row], be = (double)beta[row];
+                    const double rho = variant == 0 ? a : 1.0;
+                    const double *Sp = seg + (size_t)i * sd, *St = seg + (size_t)(i + 1) * sd;
+                    LOAD_TOKEN(t);
+                    const double *dOt = dO + row * d_v;
+                    /* r and u of this step, from S_{t-1} */
+                    for (int e = 0; e < d_v; ++e) {
+                        double s = 0.0;
+                        for (int c = 0; c < d_k; ++c) s += Sp[(size_t)e * d_k + c] * kt[c];
+                        r[e] = s;
+                        u[e] = be * (vt[e] - rho * s);
+                    }
+                    /* output o_t = S_t q_t: dq_t = S_t^T dO_t; G += dO_t q_t^T */
+                    for (int c = 0; c < d_k; ++c) {
+                        double s = 0.0;
+                        for (int e = 0; e < d_v; ++e) s += St[(size_t)e * d_k + c] * dOt[e];
+                        dq[row * d_k + c] = s;
+                    }
+                    for (int e = 0; e < d_v; ++e)
+                        for (int c = 0; c < d_k; ++c) G[(size_t)e * d_k + c] += dOt[e] * qt[c];
+                    /* S_t = alpha S_{t-1} + u k^T */
+                    double dbe = 0.0, dal = 0.0, ur = 0.0;
+                    for (int e = 0; e < d_v; ++e) {
+                        double s = 0.0;
+                        for (int c = 0; c < d_k; ++c) s += G[(size_t)e * d_k + c] * kt[c];
+                        du[e] = s;
+                        dv[row * d_v + e] = be * s;
+                        dbe += s * (vt[e] - rho * r[e]);
+                        ur += s * r[e];
+                        dr[e] = -be * rho * s;
+                    }
+                    for (size_t x = 0; x < sd; ++x) dal += G[x] * Sp[x];
+                    if (variant == 0) dal += -be * ur;
+                    dalpha[row] = dal;
+                    dbeta[row] = dbe;
+                    for (int c = 0; c < d_k; ++c) {
+                        double s = 0.0;
+                        for (int e = 0; e < d_v; ++e)
+                            s += G[(size_t)e * d_k + c] * u[e] + Sp[(size_t)e * d_k + c] * dr[e];
+                        dk[row * d_k + c] = s;
+                    }
+                    /* gradient of S_{t-1} */
+                    for (int e = 0; e < d_v; ++e)
+                        for (int c = 0; c < d_k; ++c)
+                            G[(size_t)e * d_k + c] = a * G[(size_t)e * d_k + c] + dr[e] * kt[c];
+                }
+            }
+#undef LOAD_TOKEN
+            if (dS0) memcpy(dS0 + ((size_t)b * H + h) * sd, G, sizeof(double) * sd);
+            free(ckpt);
+            free(seg);
+            free(G);
+            free(kt);
+            free(qt);
+            free(vt);
+            free(r);
+            free(u);
+            free(du);
+            free(dr);
+        }
+    }
+    return 0;
 }

@@ -541,3 +541,138 @@ def test_rope_scores_depend_only_on_relative_position():
     # and rotation is not the identity: without it the outputs differ
     plain = oracle.attention("swa", q, k, v, 1, 1, w, centred=True)
     assert np.abs(plain - base).max() > 1e-3
+
+
+# --------------------------------------------------------------------------
+# Backward pass: reverse-mode derivatives of the forward definitions
+# --------------------------------------------------------------------------
+
+def _central_difference(fn, arr, idx, eps=1e-3):
+    """d fn / d arr[idx] by a central difference taken on the float32 values the
+    oracle actually reads (the step is measured after rounding)."""
+    a = arr.copy()
+    a[idx] += eps
+    hi, f_hi = float(a[idx]), fn(a)
+    a = arr.copy()
+    a[idx] -= eps
+    lo, f_lo = float(a[idx]), fn(a)
+    return (f_hi - f_lo) / (hi - lo)
+
+
+_PROBES4 = [(0, 0, 0, 0), (0, 3, 1, 2), (0, 7, 0, 1), (0, 12, 1, 3)]
+
+
+@pytest.mark.parametrize("kind,P,dil,w,centred,rope", [
+    ("swa", 1, 1, 4, False, 0.0), ("dswa", 2, 2, 3, False, 0.0), ("swa", 1, 1, 5, True, 100.0),
+    ("dswa", 3, 2, 4, True, 10.0), ("swa", 1, 1, 30, False, 0.0)])
+def test_attention_backward_matches_central_differences(kind, P, dil, w, centred, rope):
+    q, k, v = (rnd((1, 13, 2, 4), s) for s in (1, 2, 3))
+    dO = np.random.default_rng(4).standard_normal((1, 13, 2, 4))
+    dq, dk, dv = oracle.attention_backward(kind, q, k, v, P, dil, w, dO, centred=centred,
+                                           rope_base=rope)
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for idx in _PROBES4:
+            def loss(a):
+                qq, kk, vv = {"q": (a, k, v), "k": (q, a, v), "v": (q, k, a)}[name]
+                o = oracle.attention(kind, qq, kk, vv, P, dil, w, centred=centred, rope_base=rope)
+                return float((o * dO).sum())
+            assert abs(_central_difference(loss, arr, idx) - grad[idx]) < 1e-6, (name, idx)
+
+
+def test_attention_backward_single_key_and_invariants():
+    q, k, v = (rnd((2, 20, 3, 8), s) for s in (5, 6, 7))
+    dO = np.random.default_rng(8).standard_normal((2, 20, 3, 8))
+    # w = 1: o = v, so dv = dO and nothing reaches q or k
+    dq, dk, dv = oracle.attention_backward("swa", q, k, v, 1, 1, 1, dO)
+    assert np.abs(dq).max() == 0 and np.abs(dk).max() == 0
+    np.testing.assert_allclose(dv, dO, rtol=0, atol=1e-15)
+    # softmax rows sum to one: sum_j dv_j = sum_i dO_i; logits are shift invariant
+    # per query: sum_j dk_j = 0 (each query's ds sums to zero)
+    for kind, P, dil, w in (("swa", 1, 1, 6), ("dswa", 4, 2, 5)):
+        dq, dk, dv = oracle.attention_backward(kind, q, k, v, P, dil, w, dO)
+        np.testing.assert_allclose(dv.sum(axis=1), dO.sum(axis=1), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("L", [13, 150])
+def test_gdn_backward_matches_central_differences(variant, L):
+    """L = 150 crosses the oracle's 64-step recompute segments."""
+    q = rnd((1, L, 2, 4), 11)
+    k = rnd((1, L, 2, 4), 12, normalise=True)
+    v = rnd((1, L, 2, 4), 13)
+    r = np.random.default_rng(14)
+    alpha = r.uniform(0.5, 0.99, (1, L, 2)).astype(np.float32)
+    beta = r.uniform(0.1, 0.9, (1, L, 2)).astype(np.float32)
+    S0 = r.standard_normal((1, 2, 4, 4)) * 0.3
+    dSf = r.standard_normal((1, 2, 4, 4))
+    dO = r.standard_normal((1, L, 2, 4))
+    g = oracle.gdn_backward(q, k, v, alpha, beta, dO, S0, dSf, variant)
+
+    def loss(qq=q, kk=k, vv=v, aa=alpha, bb=beta, SS=S0):
+        o, S = oracle.gdn(qq, kk, vv, aa, bb, SS, variant=variant)
+        return float((o * dO).sum() + (S * dSf).sum())
+    ts = [0, 5, L // 2, L - 1]
+    for name, arr, grad in (("qq", q, g["dq"]), ("kk", k, g["dk"]), ("vv", v, g["dv"])):
+        for t in ts:
+            idx = (0, t, t % 2, (3 * t) % 4)
+            n = _central_difference(lambda a: loss(**{name: a}), arr, idx)
+            assert abs(n - grad[idx]) < 1e-6 * (1 + abs(n)), (name, idx, n, grad[idx])
+    for name, arr, grad in (("aa", alpha, g["dalpha"]), ("bb", beta, g["dbeta"])):
+        for t in ts:
+            idx = (0, t, (t + 1) % 2)
+            n = _central_difference(lambda a: loss(**{name: a}), arr, idx, eps=1e-4)
+            assert abs(n - grad[idx]) < 1e-6 * (1 + abs(n)), (name, idx, n, grad[idx])
+    for idx in ((0, 0, 0, 0), (0, 1, 2, 3)):
+        a = S0.copy()
+        a[idx] += 1e-6
+        f_hi = loss(SS=a)
+        a[idx] -= 2e-6
+        n = (f_hi - loss(SS=a)) / 2e-6
+        assert abs(n - g["dS0"][idx]) < 1e-6 * (1 + abs(n))
+
+
+@pytest.mark.parametrize("variant", [0, 1])
+def test_gdn_backward_frozen_state_closed_form(variant):
+    """beta = 0, alpha = 1 freezes the state (S_t = S0, o_t = S0 q_t).  Then
+    dq_t = S0^T dO_t, dk = dv = 0, dS0 = dS_final + sum_t dO_t q_t^T, and with
+    G_t = dS_final + sum_{s>=t} dO_s q_s^T: dalpha_t = <G_t, S0> and
+    dbeta_t = (G_t k_t) . (v_t - S0 k_t)."""
+    B, L, H, d = 1, 9, 2, 5
+    q, v = rnd((B, L, H, d), 21), rnd((B, L, H, d), 23)
+    k = rnd((B, L, H, d), 22, normalise=True)
+    alpha = np.ones((B, L, H), np.float32)
+    beta = np.zeros((B, L, H), np.float32)
+    r = np.random.default_rng(24)
+    S0, dSf = r.standard_normal((B, H, d, d)), r.standard_normal((B, H, d, d))
+    dO = r.standard_normal((B, L, H, d))
+    g = oracle.gdn_backward(q, k, v, alpha, beta, dO, S0, dSf, variant)
+    q64, k64, v64 = (x.astype(np.float64) for x in (q, k, v))
+    np.testing.assert_allclose(g["dq"], np.einsum("bhvk,blhv->blhk", S0, dO), atol=1e-12)
+    assert np.abs(g["dk"]).max() == 0 and np.abs(g["dv"]).max() == 0
+    np.testing.assert_allclose(g["dS0"], dSf + np.einsum("blhv,blhk->bhvk", dO, q64), atol=1e-12)
+    for t in range(L):
+        G = dSf + np.einsum("blhv,blhk->bhvk", dO[:, t:], q64[:, t:])
+        np.testing.assert_allclose(g["dalpha"][:, t], np.einsum("bhvk,bhvk->bh", G, S0), atol=1e-11)
+        Gk = np.einsum("bhvk,bhk->bhv", G, k64[:, t])
+        resid = v64[:, t] - np.einsum("bhvk,bhk->bhv", S0, k64[:, t])
+        np.testing.assert_allclose(g["dbeta"][:, t], (Gk * resid).sum(-1), atol=1e-11)
+
+
+def test_layer_backward_gates_and_sum_match_central_differences():
+    wl = WORKLOADS["tiny_fp32"].with_(L=24, H=2, d_k=4, d_v=4, P=2, swa_window=5, dswa_window=3,
+                                      dilation=2)
+    inp = make_inputs(wl, seed=3)
+    dout = np.random.default_rng(5).standard_normal((1, 24, 2, 4))
+    g = oracle.backward(inp, dout)
+
+    def loss_with(**over):
+        import dataclasses
+        return float((oracle.forward(dataclasses.replace(inp, **over))["out"] * dout).sum())
+    for idx in ((0, 0), (1, 1), (0, 2), (1, 2)):
+        n = _central_difference(lambda a: loss_with(gates=a), inp.gates, idx)
+        assert abs(n - g["dgates"][idx]) < 1e-6 * (1 + abs(n))
+    # q feeds all three branches
+    for idx in ((0, 3, 0, 1), (0, 20, 1, 3)):
+        n = _central_difference(lambda a: loss_with(q=a), inp.q, idx)
+        assert abs(n - g["dq"][idx]) < 1e-6 * (1 + abs(n))
