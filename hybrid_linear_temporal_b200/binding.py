@@ -63,6 +63,7 @@ def load_library(path: str | None = None):
         "hlta_destroy": ([vp], st),
         "hlta_forward": ([vp, i, vp, vp, vp, fp, fp, fp, fp, fp, vp, u, vp], st),
         "hlta_forward_host": ([vp, i, vp, vp, vp, fp, fp, fp, fp, fp, vp, u, vp], st),
+        "hlta_backward": ([vp, i, vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, fp, u, vp], st),
         "hlta_stream_step": ([vp, i, vp, vp, vp, fp, fp, fp, vp, u, vp], st),
         "hlta_state_get": ([vp, fp, ctypes.POINTER(ctypes.c_longlong), vp], st),
         "hlta_stream_reset": ([vp, vp], st),
@@ -196,6 +197,35 @@ class HLTA:
             self.h, L, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(gates),
             _ptr(S0), _ptr(S_out), _ptr(out), branches, _stream(stream)))
         return out
+
+    def backward(self, q, k, v, alpha, beta, gates, dout, S0=None, dS_final=None, want_dS0=False,
+                 branches=BRANCH_ALL, stream=None):
+        """Gradients of ``forward`` (hlta_backward).  Returns a dict of tensors:
+        dq, dk, dv (cfg dtype), dalpha, dbeta, dgates and dS0 (float32; dS0 only
+        when want_dS0)."""
+        import torch
+        c = self.cfg
+        L = q.shape[1]
+        self._check_inputs(L, q, k, v, alpha, beta, gates)
+        dt = self._torch_dtype()
+        self._check_tensor(dout, "dout", (c.B, L, c.H, c.d_v), dt)
+        for name, s in (("S0", S0), ("dS_final", dS_final)):
+            if s is not None:
+                self._check_tensor(s, name, (c.B, c.H, c.d_v, c.d_k), torch.float32)
+        dev = q.device
+        r = {"dq": torch.empty((c.B, L, c.H, c.d_k), dtype=dt, device=dev),
+             "dk": torch.empty((c.B, L, c.H, c.d_k), dtype=dt, device=dev),
+             "dv": torch.empty((c.B, L, c.H, c.d_v), dtype=dt, device=dev),
+             "dalpha": torch.empty((c.B, L, c.H), dtype=torch.float32, device=dev),
+             "dbeta": torch.empty((c.B, L, c.H), dtype=torch.float32, device=dev),
+             "dgates": torch.empty((c.H, 3), dtype=torch.float32, device=dev),
+             "dS0": torch.empty((c.B, c.H, c.d_v, c.d_k), dtype=torch.float32, device=dev)
+             if want_dS0 else None}
+        _check(self.lib, self.lib.hlta_backward(
+            self.h, L, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(gates), _ptr(S0),
+            _ptr(dout), _ptr(dS_final), _ptr(r["dq"]), _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dalpha"]),
+            _ptr(r["dbeta"]), _ptr(r["dgates"]), _ptr(r["dS0"]), branches, _stream(stream)))
+        return r
 
     def forward_host(self, q, k, v, alpha, beta, gates, S0=None, S_out=None, out=None,
                      branches=BRANCH_ALL, stream=None):

@@ -93,6 +93,14 @@ struct hlta_handle {
     float *acc2 = nullptr;
     // rotated q and k for the attention branches (rope_base > 0)
     void *q_rot = nullptr, *k_rot = nullptr;
+    // backward scratch: one block allocated at the first hlta_backward, kept
+    char *bw_block = nullptr;
+    float *g_dq = nullptr, *g_dk = nullptr, *g_dv = nullptr, *g_dq_att = nullptr, *g_dk_att = nullptr;
+    float *g_lse = nullptr, *g_rowdot[3] = {nullptr, nullptr, nullptr};
+    float *bw_W = nullptr, *bw_TbV = nullptr, *bw_Kd = nullptr, *bw_T = nullptr, *bw_Lc = nullptr;
+    float *bw_ell = nullptr, *bw_S = nullptr, *bw_dS = nullptr, *bw_U = nullptr, *bw_ws = nullptr;
+    size_t bw_ws_floats = 0;
+    int bw_grid = 0;
     // profiling (hlta_profile_enable)
     bool prof = false;
     struct Mark {
@@ -477,6 +485,7 @@ hlta_status hlta_destroy(hlta_handle *h) {
     cudaFree(h->acc2);
     cudaFree(h->q_rot);
     cudaFree(h->k_rot);
+    cudaFree(h->bw_block);
     if (h->side) cudaStreamDestroy(h->side);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
@@ -511,6 +520,207 @@ hlta_status hlta_forward(hlta_handle *h, int L, const void *q, const void *k, co
     st = run_pass(h, in, 0, L, k, v, L, true, S0, (branches & HLTA_BRANCH_GDN) ? S_out : nullptr,
                   out, branches, s);
     if (st != HLTA_OK) return st;
+    CK(cudaGetLastError());
+    return ok();
+}
+
+namespace {
+
+// Carves the backward scratch out of one allocation (sizes for max_seq_len).
+hlta_status ensure_bwd_scratch(hlta_handle *h) {
+    if (h->bw_block) return HLTA_OK;
+    const hlta_config &c = h->cfg;
+    const size_t rows = (size_t)c.B * c.max_seq_len * c.H, bh = (size_t)c.B * c.H;
+    const size_t nc = (size_t)(c.max_seq_len + 63) / 64, ch = bh * nc;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
+    h->bw_grid = (int)(ch < (size_t)2 * sms ? ch : (size_t)2 * sms);
+    h->bw_ws_floats = hlta::gdn_bwd_ws_floats(c.d_k, c.d_v);
+    const bool rope = c.rope_base > 0.f;
+    std::vector<std::pair<float **, size_t>> parts = {
+        {&h->g_dq, rows * c.d_k}, {&h->g_dk, rows * c.d_k}, {&h->g_dv, rows * c.d_v},
+        {&h->g_dq_att, rope ? rows * c.d_k : 0}, {&h->g_dk_att, rope ? rows * c.d_k : 0},
+        {&h->g_lse, rows}, {&h->g_rowdot[0], rows}, {&h->g_rowdot[1], rows}, {&h->g_rowdot[2], rows},
+        {&h->bw_W, ch * 64 * c.d_k}, {&h->bw_TbV, ch * 64 * c.d_v}, {&h->bw_Kd, ch * 64 * c.d_k},
+        {&h->bw_T, ch * 64 * 64}, {&h->bw_Lc, ch * c.d_v * c.d_k}, {&h->bw_ell, ch * 64},
+        {&h->bw_S, ch * c.d_v * c.d_k}, {&h->bw_dS, ch * c.d_v * c.d_k}, {&h->bw_U, ch * 64 * c.d_v},
+        {&h->bw_ws, (size_t)h->bw_grid * h->bw_ws_floats}};
+    size_t total = 0;
+    for (auto &p : parts) total += (p.second * sizeof(float) + 255) / 256 * 256;
+    if (cudaMalloc((void **)&h->bw_block, total) != cudaSuccess) {
+        cudaGetLastError();
+        h->bw_block = nullptr;
+        return fail(HLTA_ERR_OOM, "hlta_backward: scratch allocation of %zu bytes failed", total);
+    }
+    size_t off = 0;
+    for (auto &p : parts) {
+        *p.first = p.second ? reinterpret_cast<float *>(h->bw_block + off) : nullptr;
+        off += (p.second * sizeof(float) + 255) / 256 * 256;
+    }
+    return HLTA_OK;
+}
+
+}  // namespace
+
+hlta_status hlta_backward(hlta_handle *h, int L, const void *q, const void *k, const void *v,
+                          const float *alpha, const float *beta, const float *gates, const float *S0,
+                          const void *dout, const float *dS_final, void *dq, void *dk, void *dv,
+                          float *dalpha, float *dbeta, float *dgates, float *dS0, unsigned branches,
+                          void *stream) {
+    INJECT("hlta_backward");
+    if (!h) return fail(HLTA_ERR_INVALID_ARG, "hlta_backward: handle is NULL");
+    const hlta_config &c = h->cfg;
+    if (L < 1 || L > c.max_seq_len)
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_backward: L=%d outside [1, max_seq_len=%d]", L, c.max_seq_len);
+    if (branches & ~7u) return fail(HLTA_ERR_INVALID_ARG, "hlta_backward: unknown branch bits");
+    if (branches == 0) branches = HLTA_BRANCH_ALL;
+    Inputs in{q, k, v, alpha, beta, gates};
+    hlta_status st = check_inputs("hlta_backward", in, dout);
+    if (st != HLTA_OK) return st;
+    const void *outs[] = {dq, dk, dv, dalpha, dbeta, dgates};
+    const char *names[] = {"dq", "dk", "dv", "dalpha", "dbeta", "dgates"};
+    for (int i = 0; i < 6; ++i) {
+        if (!outs[i]) return fail(HLTA_ERR_INVALID_ARG, "hlta_backward: %s is NULL", names[i]);
+        if (!aligned16(outs[i]))
+            return fail(HLTA_ERR_INVALID_ARG, "hlta_backward: %s is not 16-byte aligned", names[i]);
+    }
+    if ((S0 && !aligned16(S0)) || (dS_final && !aligned16(dS_final)) || (dS0 && !aligned16(dS0)))
+        return fail(HLTA_ERR_INVALID_ARG, "hlta_backward: S0/dS_final/dS0 not 16-byte aligned");
+    if ((branches & HLTA_BRANCH_GDN) && c.gdn_form != HLTA_GDN_DECAYED)
+        return fail(HLTA_ERR_UNSUPPORTED, "hlta_backward: the memory backward covers gdn_form = HLTA_GDN_DECAYED");
+    CK(cudaSetDevice(h->device));
+    st = ensure_bwd_scratch(h);
+    if (st != HLTA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = c.dtype == HLTA_BF16;
+    const size_t rows = (size_t)c.B * L * c.H;
+
+    // memory branch: stores the fp32 gradient accumulators, dalpha, dbeta
+    if (branches & HLTA_BRANCH_GDN) {
+        hlta::GdnBwdArgs a;
+        a.q = q;
+        a.k = k;
+        a.v = v;
+        a.dout = dout;
+        a.alpha = alpha;
+        a.beta = beta;
+        a.gates = gates;
+        a.S0 = S0;
+        a.dS_final = dS_final;
+        a.L = L;
+        a.B = c.B;
+        a.H = c.H;
+        a.d_k = c.d_k;
+        a.d_v = c.d_v;
+        a.bw_W = h->bw_W;
+        a.bw_TbV = h->bw_TbV;
+        a.bw_Kd = h->bw_Kd;
+        a.bw_T = h->bw_T;
+        a.bw_Lc = h->bw_Lc;
+        a.bw_ell = h->bw_ell;
+        a.bw_S = h->bw_S;
+        a.bw_dS = h->bw_dS;
+        a.bw_U = h->bw_U;
+        a.ws = h->bw_ws;
+        a.ws_per_cta = h->bw_ws_floats;
+        const long long ch = (long long)c.B * c.H * ((L + 63) / 64);
+        a.grid_chunks = (int)(ch < h->bw_grid ? ch : h->bw_grid);
+        a.dq = h->g_dq;
+        a.dk = h->g_dk;
+        a.dv = h->g_dv;
+        a.dalpha = dalpha;
+        a.dbeta = dbeta;
+        a.dS0 = dS0;
+        a.rowdot = h->g_rowdot[2];
+        CK(hlta::launch_gdn_bwd(a, bf16, s));
+    } else {
+        CK(cudaMemsetAsync(h->g_dq, 0, rows * c.d_k * sizeof(float), s));
+        CK(cudaMemsetAsync(h->g_dk, 0, rows * c.d_k * sizeof(float), s));
+        CK(cudaMemsetAsync(h->g_dv, 0, rows * c.d_v * sizeof(float), s));
+        CK(cudaMemsetAsync(dalpha, 0, rows * sizeof(float), s));
+        CK(cudaMemsetAsync(dbeta, 0, rows * sizeof(float), s));
+        if (dS0) CK(cudaMemsetAsync(dS0, 0, state_elems(c) * sizeof(float), s));
+    }
+
+    // attention branches: add into the accumulators (rotated-frame dq, dk apart)
+    const bool rope = c.rope_base > 0.f && (branches & 3u);
+    hlta::BwdFinalizeArgs fq;
+    fq.rope = rope ? 1 : 0;
+    for (int m = 0; m < 64; ++m)
+        fq.inv_freq[m] = rope && m < c.d_k / 2 ? pow((double)c.rope_base, -2.0 * m / c.d_k) : 0.0;
+    const void *qa = q, *ka = k;
+    float *adq = h->g_dq, *adk = h->g_dk;
+    if (rope) {
+        hlta::RopeArgs r;
+        r.q = q;
+        r.k = k;
+        r.q_out = h->q_rot;
+        r.k_out = h->k_rot;
+        r.B = c.B;
+        r.n = L;
+        r.H = c.H;
+        r.d = c.d_k;
+        r.pos0 = 0;
+        for (int m = 0; m < 64; ++m) r.inv_freq[m] = fq.inv_freq[m];
+        CK(hlta::launch_rope(r, bf16, s));
+        qa = h->q_rot;
+        ka = h->k_rot;
+        adq = h->g_dq_att;
+        adk = h->g_dk_att;
+        CK(cudaMemsetAsync(adq, 0, rows * c.d_k * sizeof(float), s));
+        CK(cudaMemsetAsync(adk, 0, rows * c.d_k * sizeof(float), s));
+    }
+    for (int br = 0; br < 2; ++br) {
+        if (!(branches & (1u << br))) continue;
+        hlta::AttnBwdArgs a;
+        a.q = qa;
+        a.k = ka;
+        a.v = v;
+        a.dout = dout;
+        a.L = L;
+        a.B = c.B;
+        a.H = c.H;
+        a.d_k = c.d_k;
+        a.d_v = c.d_v;
+        a.geom = window_of(c, br);
+        a.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d_k);
+        a.scale = 1.f / sqrtf((float)c.d_k);
+        a.gates = gates;
+        a.gate_col = br;
+        a.lse = h->g_lse;
+        a.rowdot = h->g_rowdot[br];
+        a.dq = adq;
+        a.dk = adk;
+        a.dv = h->g_dv;
+        CK(hlta::launch_attn_bwd(a, bf16, s));
+    }
+
+    // accumulators to the tensor type
+    fq.acc = h->g_dq;
+    fq.att = rope ? h->g_dq_att : nullptr;
+    fq.out = dq;
+    fq.rows = (long long)rows;
+    fq.d = c.d_k;
+    fq.L = L;
+    fq.H = c.H;
+    CK(hlta::launch_bwd_finalize(fq, bf16, s));
+    hlta::BwdFinalizeArgs fk = fq;
+    fk.acc = h->g_dk;
+    fk.att = rope ? h->g_dk_att : nullptr;
+    fk.out = dk;
+    CK(hlta::launch_bwd_finalize(fk, bf16, s));
+    hlta::BwdFinalizeArgs fv = fq;
+    fv.acc = h->g_dv;
+    fv.att = nullptr;
+    fv.rope = 0;
+    fv.out = dv;
+    fv.d = c.d_v;
+    CK(hlta::launch_bwd_finalize(fv, bf16, s));
+
+    // gate gradients
+    CK(cudaMemsetAsync(dgates, 0, (size_t)c.H * 3 * sizeof(float), s));
+    for (int br = 0; br < 3; ++br)
+        if (branches & (1u << br)) CK(hlta::launch_gate_grad(h->g_rowdot[br], c.B, L, c.H, br, dgates, s));
     CK(cudaGetLastError());
     return ok();
 }

@@ -80,6 +80,58 @@ struct RopeArgs {
 };
 cudaError_t launch_rope(const RopeArgs &a, bool bf16, cudaStream_t s);
 
+// Arguments of the CUDA-core attention backward (one branch).  q, k are the
+// tensors the forward branch read (rotated copies when rotary embedding is on).
+struct AttnBwdArgs {
+    const void *q, *k, *v;   // [B, L, H, d] dtype
+    const void *dout;        // [B, L, H, d_v] dtype: gradient of the layer output
+    int L, B, H, d_k, d_v;
+    WindowGeom geom;
+    float scale_log2;        // log2(e) / sqrt(d_k)
+    float scale;             // 1 / sqrt(d_k)
+    const float *gates;      // [H, 3]
+    int gate_col;            // 0 = SWA, 1 = DSWA
+    float *lse;              // [B*L*H] scratch: log2-domain log-sum-exp of the row
+    float *rowdot;           // [B*L*H] out: dout_i . o_i (the branch's ungated output)
+    float *dq, *dk, *dv;     // [B, L, H, d] fp32 accumulators (added to)
+};
+cudaError_t launch_attn_bwd(const AttnBwdArgs &a, bool bf16, cudaStream_t s);
+
+// Arguments of the chunked memory backward (gdn_bwd.cu).  Inputs [B, L, H, d]
+// dtype, alpha/beta [B, L, H]; chunk-indexed scratch [B*H, nc, ...] fp32 with
+// nc = ceil(L / 64); ws: grid_chunks per-CTA workspaces of ws_per_cta floats.
+struct GdnBwdArgs {
+    const void *q, *k, *v, *dout;
+    const float *alpha, *beta, *gates;
+    const float *S0;        // [B, H, d_v, d_k] or nullptr (zeros)
+    const float *dS_final;  // [B, H, d_v, d_k] or nullptr (zeros)
+    int L, B, H, d_k, d_v;
+    float *bw_W, *bw_TbV, *bw_Kd, *bw_T, *bw_Lc, *bw_ell, *bw_S, *bw_dS, *bw_U;
+    float *ws;
+    size_t ws_per_cta;
+    int grid_chunks;
+    float *dq, *dk, *dv;    // [B, L, H, d] fp32: stored (the attention branches add after)
+    float *dalpha, *dbeta;  // [B, L, H]
+    float *dS0;             // [B, H, d_v, d_k] or nullptr
+    float *rowdot;          // [B*L*H]: dout . o of the memory branch
+};
+size_t gdn_bwd_ws_floats(int d_k, int d_v);
+cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, bool bf16, cudaStream_t s);
+
+// out = acc + R^T att (R: the rotary embedding when rope, else identity; att may
+// be null), converted to the tensor type.  Rows are (b, t, h) with t < L.
+struct BwdFinalizeArgs {
+    const float *acc, *att;
+    void *out;
+    long long rows;
+    int d, L, H;
+    int rope;
+    double inv_freq[64];
+};
+cudaError_t launch_bwd_finalize(const BwdFinalizeArgs &a, bool bf16, cudaStream_t s);
+// dgates[h*3 + col] = sum over (b, t) of rowdot[(b*L + t)*H + h]
+cudaError_t launch_gate_grad(const float *rowdot, int B, int L, int H, int col, float *dgates, cudaStream_t s);
+
 // Sets the thread-local message returned by hlta_last_error() (empty clears it).
 void set_last_error(const char *msg);
 

@@ -148,6 +148,32 @@ HLTA_API hlta_status hlta_forward(hlta_handle *h, int L, const void *q, const vo
                          void *stream);
 
 /*
+ * hlta_backward: gradients of hlta_forward (the same L, inputs, S0 and branch
+ * selection) for training.  The pages train the layer but print no backward;
+ * this is the chain rule through section 2.2.1's recurrence (memory branch,
+ * chunk form), section 2.2.2's Eq. (7)/(8) softmax windows and the per-head
+ * gated sum.
+ *   dout:     [B,L,H,d_v] cfg.dtype, the gradient of the layer output.
+ *   dS_final: [B,H,d_v,d_k] float32 gradient of the final memory state, or NULL
+ *             (zero).
+ *   dq, dk:   [B,L,H,d_k] cfg.dtype, dv: [B,L,H,d_v] cfg.dtype (written).
+ *   dalpha, dbeta: [B,L,H] float32 (written; zero without the memory branch).
+ *   dgates:   [H,3] float32 (written; zero in unselected columns).
+ *   dS0:      [B,H,d_v,d_k] float32 gradient of the initial state, or NULL.
+ * The forward is recomputed inside (nothing is kept from hlta_forward).
+ * Scratch (about 7 x B*max_seq_len*H*128 floats plus 4 states per 64-token
+ * chunk) is allocated at the first call and kept until hlta_destroy
+ * (HLTA_ERR_OOM when it cannot be).  The memory branch's backward covers
+ * gdn_form = HLTA_GDN_DECAYED (HLTA_ERR_UNSUPPORTED otherwise).  Centred
+ * windows and rotary embedding are covered.  Enqueued on `stream`.
+ */
+HLTA_API hlta_status hlta_backward(hlta_handle *h, int L, const void *q, const void *k, const void *v,
+                                   const float *alpha, const float *beta, const float *gates,
+                                   const float *S0, const void *dout, const float *dS_final, void *dq,
+                                   void *dk, void *dv, float *dalpha, float *dbeta, float *dgates,
+                                   float *dS0, unsigned branches, void *stream);
+
+/*
  * hlta_forward_host: hlta_forward on HOST buffers (pinned memory recommended):
  * copies the inputs to device staging owned by the handle (allocated at the
  * first call, kept until hlta_destroy), runs the layer, copies `out` (and
