@@ -29,7 +29,7 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-from workloads import WORKLOADS, make_inputs, algorithmic_work  # noqa: E402
+from workloads import WORKLOADS, make_inputs, algorithmic_work, backward_work  # noqa: E402
 
 METRIC = "hybrid temporal attention fwd tokens/s at L=32760 bf16; % of roofline"
 L2_BYTES = 126 * 2 ** 20
@@ -47,6 +47,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     return ap.parse_args()
 
 
@@ -329,6 +330,53 @@ def attention_alone(layer, d, out, stream, reps=5):
     return sw["total_ms"] / sw["passes"], ds["total_ms"] / ds["passes"]
 
 
+# FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+# (the SM count and maximum clock of the B200s measured here).
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_measure(layer, d, wl, stream, steps, world):
+    """Device time of hlta_backward (whole layer, then the attention branches and
+    the memory branch alone), CUDA events on the launching stream."""
+    import torch
+    from hybrid_linear_temporal_b200 import BRANCH_SWA, BRANCH_DSWA, BRANCH_GDN, BRANCH_ALL
+    g = torch.Generator(device="cpu").manual_seed(7)
+    dout = torch.randn((wl.B, wl.L, wl.H, wl.d_v), generator=g).to(d["q"].dtype).cuda()
+
+    def timed(branches, n):
+        layer.backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["gates"], dout,
+                       branches=branches, stream=stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            layer.backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["gates"], dout,
+                           branches=branches, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1) / n, world)
+
+    ms = timed(BRANCH_ALL, steps)
+    ms_att = timed(BRANCH_SWA | BRANCH_DSWA, 1)
+    ms_mem = timed(BRANCH_GDN, 1)
+    work = backward_work(wl)
+    att_flops = work["swa_flops"] + work["dswa_flops"]
+    ach = att_flops / (ms_att * 1e-3) / 1e12
+    mem_ach = work["gdn_flops"] / (ms_mem * 1e-3) / 1e12
+    return {"ms_per_step": round(ms, 3), "steps": steps,
+            "tokens_per_s": round(world * wl.B * wl.L / (ms * 1e-3), 1),
+            "ms_attention": round(ms_att, 3), "ms_memory": round(ms_mem, 3),
+            "roofline": {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
+                         "achieved": round(ach, 2), "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                         "frac": round(ach / FP32_PEAK_TFLOPS, 4), "traffic": None,
+                         "algorithmic": {"flops": att_flops, "rule": "10*d flops per in-band (query, key) pair"},
+                         "peak_kind": "fp32 FMA of the CUDA cores, derived: 148 SMs x 128 lanes x 2 x 1.965 GHz"},
+            "memory": {"achieved_tflops": round(mem_ach, 2), "frac_of_fp32": round(mem_ach / FP32_PEAK_TFLOPS, 4),
+                       "algorithmic_flops": work["gdn_flops"],
+                       "rule": "chunk form: 32*C^2*d + 22*C*d^2 + (2/3)*C^3 per chunk"},
+            "dtype": "fp32 arithmetic, bf16 tensors"}
+
+
 def run_ours(args, world, rank, local):
     import torch
     from hybrid_linear_temporal_b200 import HLTA, build
@@ -429,6 +477,10 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.nbytes),
                "ms_per_step": round(ms_e2e, 3), "steps": n_e2e}
 
+    bwd = None
+    if not args.no_backward:
+        bwd = backward_measure(layer, d, wl, stream, max(1, min(args.steps, 3)), world)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, args.cpu_seconds)
@@ -444,7 +496,7 @@ def run_ours(args, world, rank, local):
                 "branches": branches,
                 "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(prof.get("kernel_launches", 0)),
-                "clocks": clk}
+                "clocks": clk, "backward": bwd}
         print(json.dumps(line), flush=True)
     layer.close()
 

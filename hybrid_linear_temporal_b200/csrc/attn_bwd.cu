@@ -13,7 +13,9 @@
 // row's softmax statistics and output, stores lse_i and dout_i.o_i, and
 // accumulates dq_i; and a key-major one (one warp per key row) that walks the
 // queries whose window admits the key (the transposed window: backward reach
-// w_hi + 1, forward reach w - 1) and accumulates dk_j and dv_j.  fp32 math.
+// w_hi + 1, forward reach w - 1) and accumulates dk_j and dv_j.  A warp reads
+// each row with one vector load (lane l holds d/32 consecutive elements) and
+// reduces eight dot products at a time with shuffles.  fp32 math.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -46,33 +48,74 @@ __device__ __forceinline__ void for_each_run(const WindowGeom &g, long long p, l
     }
 }
 
-template <typename T, int DK>
-__device__ __forceinline__ float dot_row(const T *x, const float *y) {
-    float acc = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < DK; ++c) acc = fmaf(to_f32(x[c]), y[c], acc);
-    return acc;
+// Row access, warp-cooperative: lane l holds elements [l*E, l*E + E) of a row
+// (E = d/32), read with one vector load, so a warp reads a whole row at once.
+template <typename T, int E>
+__device__ __forceinline__ void load_part(const T *row, int lane, float (&x)[E]) {
+    if constexpr (sizeof(T) == 2) {
+        if constexpr (E == 4) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(row + lane * 4);
+            const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+            const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
+            x[0] = __low2float(a);
+            x[1] = __high2float(a);
+            x[2] = __low2float(b);
+            x[3] = __high2float(b);
+        } else {
+            const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(row + lane * 2);
+            x[0] = __low2float(a);
+            x[1] = __high2float(a);
+        }
+    } else {
+        if constexpr (E == 4) {
+            const float4 u = *reinterpret_cast<const float4 *>(row + lane * 4);
+            x[0] = u.x;
+            x[1] = u.y;
+            x[2] = u.z;
+            x[3] = u.w;
+        } else {
+            const float2 u = *reinterpret_cast<const float2 *>(row + lane * 2);
+            x[0] = u.x;
+            x[1] = u.y;
+        }
+    }
 }
+
+template <int E>
+__device__ __forceinline__ float part_dot(const float (&a)[E], const float (&b)[E]) {
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) s = fmaf(a[e], b[e], s);
+    return s;
+}
+
+// Reduces G independent per-lane partial sums across the warp (all lanes get
+// every sum).
+template <int G>
+__device__ __forceinline__ void warp_sum_n(float (&x)[G]) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) x[g] += __shfl_xor_sync(0xffffffffu, x[g], o);
+}
+
+constexpr int kGrp = 8;  // keys (or queries) handled per group
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(128) attn_bwd_q_kernel(AttnBwdArgs a) {
-    constexpr int OK_ = DK / 32, OV = DV / 32;
-    __shared__ float q_sh[4][DK];
-    __shared__ float do_sh[4][DV];
+    constexpr int EK = DK / 32, EV = DV / 32;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const long long row = (long long)blockIdx.x * 4 + wid;
     const long long total = (long long)a.B * a.L * a.H;
-    const bool live = row < total;
-    const long long rr = live ? row : 0;
-    const int h = (int)(rr % a.H);
-    const long long i = (rr / a.H) % a.L;
-    const int b = (int)(rr / ((long long)a.H * a.L));
-    const T *qp = static_cast<const T *>(a.q) + (size_t)rr * DK;
-    const T *dp_ = static_cast<const T *>(a.dout) + (size_t)rr * DV;
-    for (int c = lane; c < DK; c += 32) q_sh[wid][c] = to_f32(qp[c]) * a.scale_log2;
-    for (int c = lane; c < DV; c += 32) do_sh[wid][c] = to_f32(dp_[c]);
-    __syncwarp();
-    if (!live) return;
+    if (row >= total) return;
+    const int h = (int)(row % a.H);
+    const long long i = (row / a.H) % a.L;
+    const int b = (int)(row / ((long long)a.H * a.L));
+    float q[EK], dO[EV];
+    load_part<T, EK>(static_cast<const T *>(a.q) + (size_t)row * DK, lane, q);
+    load_part<T, EV>(static_cast<const T *>(a.dout) + (size_t)row * DV, lane, dO);
+#pragma unroll
+    for (int e = 0; e < EK; ++e) q[e] *= a.scale_log2;
 
     const T *kb = static_cast<const T *>(a.k) + (size_t)b * a.L * a.H * DK;
     const T *vb = static_cast<const T *>(a.v) + (size_t)b * a.L * a.H * DV;
@@ -80,124 +123,146 @@ __global__ void __launch_bounds__(128) attn_bwd_q_kernel(AttnBwdArgs a) {
     auto vrow = [&](long long p) { return vb + ((size_t)p * a.H + h) * DV; };
 
     // pass 1: softmax statistics and the branch output o_i (online, log2 domain)
-    float m_run = -INFINITY, l_run = 0.f, o[OV];
+    float m_run = -INFINITY, l_run = 0.f, o[EV];
 #pragma unroll
-    for (int c = 0; c < OV; ++c) o[c] = 0.f;
+    for (int e = 0; e < EV; ++e) o[e] = 0.f;
     for_each_run(a.geom, i, a.L, [&](long long p0, int cnt) {
-        const bool act = lane < cnt;
-        const float x = act ? dot_row<T, DK>(krow(p0 + lane), q_sh[wid]) : -INFINITY;
-        const float m_new = fmaxf(m_run, warp_max(x));
-        const float corr = exp2f(m_run - m_new);
-        const float pj = act ? exp2f(x - m_new) : 0.f;
-        l_run = l_run * corr + warp_sum(pj);
+        for (int j0 = 0; j0 < cnt; j0 += kGrp) {
+            float x[kGrp], vv[kGrp][EV];
 #pragma unroll
-        for (int c = 0; c < OV; ++c) o[c] *= corr;
-        for (int j = 0; j < cnt; ++j) {
-            const float pjj = __shfl_sync(0xffffffffu, pj, j);
-            const T *vp = vrow(p0 + j);
+            for (int g = 0; g < kGrp; ++g) {
+                float kk[EK];
+                const long long p = p0 + min(j0 + g, cnt - 1);
+                load_part<T, EK>(krow(p), lane, kk);
+                load_part<T, EV>(vrow(p), lane, vv[g]);
+                x[g] = part_dot<EK>(q, kk);
+            }
+            warp_sum_n<kGrp>(x);
+            float mx = m_run;
 #pragma unroll
-            for (int c = 0; c < OV; ++c) o[c] = fmaf(pjj, to_f32(vp[lane + 32 * c]), o[c]);
+            for (int g = 0; g < kGrp; ++g) {
+                if (j0 + g >= cnt) x[g] = -INFINITY;
+                mx = fmaxf(mx, x[g]);
+            }
+            const float corr = exp2f(m_run - mx);
+            l_run *= corr;
+#pragma unroll
+            for (int e = 0; e < EV; ++e) o[e] *= corr;
+#pragma unroll
+            for (int g = 0; g < kGrp; ++g) {
+                const float p = exp2f(x[g] - mx);
+                l_run += p;
+#pragma unroll
+                for (int e = 0; e < EV; ++e) o[e] = fmaf(p, vv[g][e], o[e]);
+            }
+            m_run = mx;
         }
-        m_run = m_new;
     });
-    float part = 0.f;
-#pragma unroll
-    for (int c = 0; c < OV; ++c) part = fmaf(o[c], do_sh[wid][lane + 32 * c], part);
-    const float rowdot = warp_sum(part) / l_run;  // dout_i . o_i
+    float rd[1] = {part_dot<EV>(o, dO)};
+    warp_sum_n<1>(rd);
+    const float rowdot = rd[0] / l_run;  // dout_i . o_i
     const float lse = m_run + log2f(l_run);
     if (lane == 0) {
-        a.lse[rr] = lse;
-        a.rowdot[rr] = rowdot;
+        a.lse[row] = lse;
+        a.rowdot[row] = rowdot;
     }
-    const float g = a.gates[h * 3 + a.gate_col];
-    const float delta = g * rowdot;
+    const float gt = a.gates[h * 3 + a.gate_col];
+    const float delta = gt * rowdot;
 
-    // pass 2: dq_i
-    float dq[OK_];
+    // pass 2: dq_i = sum_j p_ij (g dout_i . v_j - delta_i) k_j / sqrt(d_k)
+    float dq[EK];
 #pragma unroll
-    for (int c = 0; c < OK_; ++c) dq[c] = 0.f;
+    for (int e = 0; e < EK; ++e) dq[e] = 0.f;
     for_each_run(a.geom, i, a.L, [&](long long p0, int cnt) {
-        float ds = 0.f;
-        if (lane < cnt) {
-            const float x = dot_row<T, DK>(krow(p0 + lane), q_sh[wid]);
-            const float p = exp2f(x - lse);
-            const float dpv = g * dot_row<T, DV>(vrow(p0 + lane), do_sh[wid]);
-            ds = p * (dpv - delta);
-        }
-        for (int j = 0; j < cnt; ++j) {
-            const float dsj = __shfl_sync(0xffffffffu, ds, j);
-            const T *kp = krow(p0 + j);
+        for (int j0 = 0; j0 < cnt; j0 += kGrp) {
+            float kk[kGrp][EK], sx[2 * kGrp];
 #pragma unroll
-            for (int c = 0; c < OK_; ++c) dq[c] = fmaf(dsj, to_f32(kp[lane + 32 * c]), dq[c]);
+            for (int g = 0; g < kGrp; ++g) {
+                float vv[EV];
+                const long long p = p0 + min(j0 + g, cnt - 1);
+                load_part<T, EK>(krow(p), lane, kk[g]);
+                load_part<T, EV>(vrow(p), lane, vv);
+                sx[g] = part_dot<EK>(q, kk[g]);
+                sx[kGrp + g] = part_dot<EV>(dO, vv);
+            }
+            warp_sum_n<2 * kGrp>(sx);
+#pragma unroll
+            for (int g = 0; g < kGrp; ++g) {
+                const float ds = j0 + g < cnt ? exp2f(sx[g] - lse) * (gt * sx[kGrp + g] - delta) : 0.f;
+#pragma unroll
+                for (int e = 0; e < EK; ++e) dq[e] = fmaf(ds, kk[g][e], dq[e]);
+            }
         }
     });
-    float *dqp = a.dq + (size_t)rr * DK;
+    float *dqp = a.dq + (size_t)row * DK + lane * EK;
 #pragma unroll
-    for (int c = 0; c < OK_; ++c) dqp[lane + 32 * c] += dq[c] * a.scale;
+    for (int e = 0; e < EK; ++e) dqp[e] += dq[e] * a.scale;
 }
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(128) attn_bwd_kv_kernel(AttnBwdArgs a) {
-    constexpr int OK_ = DK / 32, OV = DV / 32;
-    __shared__ float k_sh[4][DK];
-    __shared__ float v_sh[4][DV];
+    constexpr int EK = DK / 32, EV = DV / 32;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const long long row = (long long)blockIdx.x * 4 + wid;
     const long long total = (long long)a.B * a.L * a.H;
-    const bool live = row < total;
-    const long long rr = live ? row : 0;
-    const int h = (int)(rr % a.H);
-    const long long j = (rr / a.H) % a.L;
-    const int b = (int)(rr / ((long long)a.H * a.L));
-    const T *kp = static_cast<const T *>(a.k) + (size_t)rr * DK;
-    const T *vp = static_cast<const T *>(a.v) + (size_t)rr * DV;
-    for (int c = lane; c < DK; c += 32) k_sh[wid][c] = to_f32(kp[c]) * a.scale_log2;
-    for (int c = lane; c < DV; c += 32) v_sh[wid][c] = to_f32(vp[c]);
-    __syncwarp();
-    if (!live) return;
+    if (row >= total) return;
+    const int h = (int)(row % a.H);
+    const long long j = (row / a.H) % a.L;
+    const int b = (int)(row / ((long long)a.H * a.L));
+    float k[EK], v[EV];
+    load_part<T, EK>(static_cast<const T *>(a.k) + (size_t)row * DK, lane, k);
+    load_part<T, EV>(static_cast<const T *>(a.v) + (size_t)row * DV, lane, v);
+#pragma unroll
+    for (int e = 0; e < EK; ++e) k[e] *= a.scale_log2;
 
     const size_t base_row = (size_t)b * a.L * a.H;
     const T *qb = static_cast<const T *>(a.q) + base_row * DK;
     const T *db = static_cast<const T *>(a.dout) + base_row * DV;
-    const float g = a.gates[h * 3 + a.gate_col];
+    const float gt = a.gates[h * 3 + a.gate_col];
     // queries whose window admits this key: r_k - w_hi <= r_q <= r_k + w - 1
-    WindowGeom gt = a.geom;
-    gt.w = a.geom.w_hi + 1;
-    gt.w_hi = a.geom.w - 1;
+    WindowGeom wt = a.geom;
+    wt.w = a.geom.w_hi + 1;
+    wt.w_hi = a.geom.w - 1;
 
-    float dk[OK_], dv[OV];
+    float dk[EK], dv[EV];
 #pragma unroll
-    for (int c = 0; c < OK_; ++c) dk[c] = 0.f;
+    for (int e = 0; e < EK; ++e) dk[e] = 0.f;
 #pragma unroll
-    for (int c = 0; c < OV; ++c) dv[c] = 0.f;
-    for_each_run(gt, j, a.L, [&](long long p0, int cnt) {
-        float p = 0.f, ds = 0.f;
-        if (lane < cnt) {
-            const long long qi = p0 + lane;
-            const size_t qrow = (size_t)qi * a.H + h;
-            const float x = dot_row<T, DK>(qb + qrow * DK, k_sh[wid]);
-            p = exp2f(x - a.lse[base_row + qrow]);
-            const float dpv = g * dot_row<T, DV>(db + qrow * DV, v_sh[wid]);
-            ds = p * (dpv - g * a.rowdot[base_row + qrow]);
-        }
-        for (int jj = 0; jj < cnt; ++jj) {
-            const float pg = g * __shfl_sync(0xffffffffu, p, jj);
-            const float dsj = __shfl_sync(0xffffffffu, ds, jj);
-            const size_t qrow = (size_t)(p0 + jj) * a.H + h;
-            const T *qp = qb + qrow * DK;
-            const T *dop = db + qrow * DV;
+    for (int e = 0; e < EV; ++e) dv[e] = 0.f;
+    for_each_run(wt, j, a.L, [&](long long p0, int cnt) {
+        for (int j0 = 0; j0 < cnt; j0 += kGrp) {
+            float qq[kGrp][EK], dd[kGrp][EV], sx[2 * kGrp];
+            float lse[kGrp], rdt[kGrp];
 #pragma unroll
-            for (int c = 0; c < OK_; ++c) dk[c] = fmaf(dsj, to_f32(qp[lane + 32 * c]), dk[c]);
+            for (int g = 0; g < kGrp; ++g) {
+                const size_t qrow = (size_t)(p0 + min(j0 + g, cnt - 1)) * a.H + h;
+                load_part<T, EK>(qb + qrow * DK, lane, qq[g]);
+                load_part<T, EV>(db + qrow * DV, lane, dd[g]);
+                lse[g] = a.lse[base_row + qrow];
+                rdt[g] = a.rowdot[base_row + qrow];
+                sx[g] = part_dot<EK>(qq[g], k);
+                sx[kGrp + g] = part_dot<EV>(dd[g], v);
+            }
+            warp_sum_n<2 * kGrp>(sx);
 #pragma unroll
-            for (int c = 0; c < OV; ++c) dv[c] = fmaf(pg, to_f32(dop[lane + 32 * c]), dv[c]);
+            for (int g = 0; g < kGrp; ++g) {
+                const bool act = j0 + g < cnt;
+                const float p = act ? exp2f(sx[g] - lse[g]) : 0.f;
+                const float ds = p * gt * (sx[kGrp + g] - rdt[g]);
+                const float pg = p * gt;
+#pragma unroll
+                for (int e = 0; e < EK; ++e) dk[e] = fmaf(ds, qq[g][e], dk[e]);
+#pragma unroll
+                for (int e = 0; e < EV; ++e) dv[e] = fmaf(pg, dd[g][e], dv[e]);
+            }
         }
     });
-    float *dkp = a.dk + (size_t)rr * DK;
-    float *dvp = a.dv + (size_t)rr * DV;
+    float *dkp = a.dk + (size_t)row * DK + lane * EK;
+    float *dvp = a.dv + (size_t)row * DV + lane * EV;
 #pragma unroll
-    for (int c = 0; c < OK_; ++c) dkp[lane + 32 * c] += dk[c] * a.scale;
+    for (int e = 0; e < EK; ++e) dkp[e] += dk[e] * a.scale;
 #pragma unroll
-    for (int c = 0; c < OV; ++c) dvp[lane + 32 * c] += dv[c];
+    for (int e = 0; e < EV; ++e) dvp[e] += dv[e];
 }
 
 template <typename T>

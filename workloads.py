@@ -199,6 +199,27 @@ def dswa_pairs(L: int, P: int, w: int, dilation: int) -> int:
     return tot
 
 
+def backward_work(wl: Workload) -> dict:
+    """Flops and HBM bytes of one backward pass of ``wl`` (all three branches).
+
+    Attention: 10 * d flops per in-band (query, key) pair (the logits again,
+    dO.v, and the three products for dq, dk, dv).  Memory branch, chunk form per
+    chunk of C tokens: 32*C^2*d + 22*C*d^2 + (2/3)*C^3 (the products of the
+    per-chunk prep, the two state scans and the token gradients).
+    Bytes: q, k, v, dout read, dq, dk, dv written, alpha, beta, dalpha, dbeta.
+    """
+    eb = 2 if wl.dtype == "bf16" else 4
+    d = wl.d_k
+    B, H, L, C = wl.B, wl.H, wl.L, wl.chunk
+    swa = 10 * d * band_pairs(L, wl.swa_window) * B * H
+    dswa = 10 * d * dswa_pairs(L, wl.P, wl.dswa_window, wl.dilation) * B * H
+    nch = math.ceil(L / C)
+    gdn = nch * (32 * C * C * d + 22 * C * d * d + (2 * C ** 3) // 3) * B * H
+    bytes_ = B * L * H * (7 * d * eb + 16)
+    return {"swa_flops": swa, "dswa_flops": dswa, "gdn_flops": gdn, "flops": swa + dswa + gdn,
+            "bytes": bytes_}
+
+
 def algorithmic_work(wl: Workload) -> dict:
     """Flops and HBM bytes the method needs for one forward pass of ``wl``.
 
