@@ -357,24 +357,29 @@ def backward_measure(layer, d, wl, stream, steps, world):
         return max_over_ranks(e0.elapsed_time(e1) / n, world)
 
     ms = timed(BRANCH_ALL, steps)
-    ms_att = timed(BRANCH_SWA | BRANCH_DSWA, 1)
-    ms_mem = timed(BRANCH_GDN, 1)
+    ms_att = timed(BRANCH_SWA | BRANCH_DSWA, 2)
+    ms_mem = timed(BRANCH_GDN, 2)
     work = backward_work(wl)
     att_flops = work["swa_flops"] + work["dswa_flops"]
     ach = att_flops / (ms_att * 1e-3) / 1e12
     mem_ach = work["gdn_flops"] / (ms_mem * 1e-3) / 1e12
+    peak = measured_peaks()["bf16_tflops_sustained"]
     return {"ms_per_step": round(ms, 3), "steps": steps,
             "tokens_per_s": round(world * wl.B * wl.L / (ms * 1e-3), 1),
             "ms_attention": round(ms_att, 3), "ms_memory": round(ms_mem, 3),
-            "roofline": {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
-                         "achieved": round(ach, 2), "peak": round(FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
-                         "frac": round(ach / FP32_PEAK_TFLOPS, 4), "traffic": None,
+            "roofline": {"kernel": "attn_bwd_dq_kernel + attn_bwd_dkv_kernel (tcgen05)", "bound": "tensor",
+                         "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(ach / peak, 4), "traffic": None,
                          "algorithmic": {"flops": att_flops, "rule": "10*d flops per in-band (query, key) pair"},
-                         "peak_kind": "fp32 FMA of the CUDA cores, derived: 148 SMs x 128 lanes x 2 x 1.965 GHz"},
-            "memory": {"achieved_tflops": round(mem_ach, 2), "frac_of_fp32": round(mem_ach / FP32_PEAK_TFLOPS, 4),
-                       "algorithmic_flops": work["gdn_flops"],
-                       "rule": "chunk form: 32*C^2*d + 22*C*d^2 + (2/3)*C^3 per chunk"},
-            "dtype": "fp32 arithmetic, bf16 tensors"}
+                         "timing": "attention branches' whole backward: the forward recompute (log-sum-exp and "
+                                   "output), dout . o, dQ and dK/dV launches",
+                         "peak_kind": "bf16 dense, sustained, measured"},
+            "memory": {"kernels": "gdn_bwd_prep, gdn_bwd_fscan, gdn_bwd_dscan, gdn_bwd_local (CUDA cores, fp32)",
+                       "bound": "alu", "achieved_tflops": round(mem_ach, 2), "peak": round(FP32_PEAK_TFLOPS, 1),
+                       "frac": round(mem_ach / FP32_PEAK_TFLOPS, 4), "algorithmic_flops": work["gdn_flops"],
+                       "rule": "chunk form: 32*C^2*d + 22*C*d^2 + (2/3)*C^3 per chunk",
+                       "peak_kind": "fp32 FMA of the CUDA cores, derived: 148 SMs x 128 lanes x 2 x 1.965 GHz"},
+            "dtype": "bf16 tensors; attention on bf16 tensor cores, memory branch in fp32"}
 
 
 def run_ours(args, world, rank, local):

@@ -56,7 +56,38 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const float *rowdot, int
     }
 }
 
+// rowdot = dout . o per (b, t, h) row, in [B, L, H] and [B, H, L] order; one warp per row.
+template <typename T>
+__global__ void __launch_bounds__(256) rowdot_kernel(const T *dout, const float *o, long long rows, int d, int L,
+                                                     int H, float *rowdot, float *rowdot_hm) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float s = 0.f;
+    for (int c = lane; c < d; c += 32) s = fmaf(to_f32(dout[row * d + c]), o[row * d + c], s);
+    s = warp_sum(s);
+    if (lane == 0) {
+        const int h = (int)(row % H);
+        const long long t = (row / H) % L, b = row / ((long long)H * L);
+        rowdot[row] = s;
+        rowdot_hm[(b * H + h) * L + t] = s;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_rowdot(const void *dout, const float *o, long long rows, int d, int L, int H, bool bf16,
+                          float *rowdot, float *rowdot_hm, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    if (bf16)
+        rowdot_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(dout), o, rows, d, L,
+                                                             H, rowdot, rowdot_hm);
+    else
+        rowdot_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float *>(dout), o, rows, d, L, H, rowdot,
+                                                    rowdot_hm);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_finalize(const BwdFinalizeArgs &a, bool bf16, cudaStream_t s) {
     if (a.rows == 0) return cudaSuccess;

@@ -16,6 +16,7 @@
 #include "hlta.h"
 #include "kernels.h"
 #include "tc_attention.h"
+#include "tc_attn_bwd.h"
 #include "tc_gdn.h"
 
 namespace {
@@ -96,7 +97,9 @@ struct hlta_handle {
     // backward scratch: one block allocated at the first hlta_backward, kept
     char *bw_block = nullptr;
     float *g_dq = nullptr, *g_dk = nullptr, *g_dv = nullptr, *g_dq_att = nullptr, *g_dk_att = nullptr;
-    float *g_lse = nullptr, *g_rowdot[3] = {nullptr, nullptr, nullptr};
+    float *g_lse = nullptr, *g_rowdot[3] = {nullptr, nullptr, nullptr}, *g_rowdot_hm = nullptr;
+    float *g_ones = nullptr;  // [H, 3] gates of one: the forward writes the ungated branch output
+    hlta::TcAttnBwd *tc_bwd = nullptr;
     float *bw_W = nullptr, *bw_TbV = nullptr, *bw_Kd = nullptr, *bw_T = nullptr, *bw_Lc = nullptr;
     float *bw_ell = nullptr, *bw_S = nullptr, *bw_dS = nullptr, *bw_U = nullptr, *bw_ws = nullptr;
     size_t bw_ws_floats = 0;
@@ -496,6 +499,7 @@ hlta_status hlta_destroy(hlta_handle *h) {
     for (auto e : h->event_pool) cudaEventDestroy(e);
     delete h->tc_attn;
     delete h->tc_gdn;
+    delete h->tc_bwd;
     delete h;
     return ok();
 }
@@ -541,6 +545,7 @@ hlta_status ensure_bwd_scratch(hlta_handle *h) {
         {&h->g_dq, rows * c.d_k}, {&h->g_dk, rows * c.d_k}, {&h->g_dv, rows * c.d_v},
         {&h->g_dq_att, rope ? rows * c.d_k : 0}, {&h->g_dk_att, rope ? rows * c.d_k : 0},
         {&h->g_lse, rows}, {&h->g_rowdot[0], rows}, {&h->g_rowdot[1], rows}, {&h->g_rowdot[2], rows},
+        {&h->g_rowdot_hm, rows}, {&h->g_ones, (size_t)c.H * 3},
         {&h->bw_W, ch * 64 * c.d_k}, {&h->bw_TbV, ch * 64 * c.d_v}, {&h->bw_Kd, ch * 64 * c.d_k},
         {&h->bw_T, ch * 64 * 64}, {&h->bw_Lc, ch * c.d_v * c.d_k}, {&h->bw_ell, ch * 64},
         {&h->bw_S, ch * c.d_v * c.d_k}, {&h->bw_dS, ch * c.d_v * c.d_k}, {&h->bw_U, ch * 64 * c.d_v},
@@ -557,6 +562,9 @@ hlta_status ensure_bwd_scratch(hlta_handle *h) {
         *p.first = p.second ? reinterpret_cast<float *>(h->bw_block + off) : nullptr;
         off += (p.second * sizeof(float) + 255) / 256 * 256;
     }
+    std::vector<float> ones((size_t)c.H * 3, 1.f);
+    CK(cudaMemcpy(h->g_ones, ones.data(), ones.size() * sizeof(float), cudaMemcpyHostToDevice));
+    h->tc_bwd = hlta::TcAttnBwd::create(c);
     return HLTA_OK;
 }
 
@@ -672,6 +680,23 @@ hlta_status hlta_backward(hlta_handle *h, int L, const void *q, const void *k, c
     }
     for (int br = 0; br < 2; ++br) {
         if (!(branches & (1u << br))) continue;
+        const hlta::WindowGeom geo = window_of(c, br);
+        if (h->tc_attn && h->tc_bwd && h->tc_bwd->covers(L, geo)) {
+            // tensor cores: the forward (ungated output and log-sum-exp), dout . o, then dQ and dK/dV
+            bool done = false;
+            cudaError_t e = h->tc_attn->run(qa, ka, v, L, geo, h->g_ones, br, hlta::OUT_STORE, h->acc, nullptr,
+                                            nullptr, h->dev_err, s, &done, h->g_lse);
+            if (e != cudaSuccess) return fail(HLTA_ERR_CUDA, "hlta_backward: forward: %s", cudaGetErrorString(e));
+            if (done) {
+                CK(hlta::launch_rowdot(dout, h->acc, (long long)rows, c.d_v, L, c.H, bf16, h->g_rowdot[br],
+                                       h->g_rowdot_hm, s));
+                e = h->tc_bwd->run(qa, ka, v, dout, L, geo, gates, br, h->g_lse, h->g_rowdot_hm, adq, adk, h->g_dv,
+                                   h->dev_err, s);
+                if (e != cudaSuccess)
+                    return fail(HLTA_ERR_CUDA, "hlta_backward: tensor-core attention: %s", cudaGetErrorString(e));
+                continue;
+            }
+        }
         hlta::AttnBwdArgs a;
         a.q = qa;
         a.k = ka;
@@ -682,7 +707,7 @@ hlta_status hlta_backward(hlta_handle *h, int L, const void *q, const void *k, c
         a.H = c.H;
         a.d_k = c.d_k;
         a.d_v = c.d_v;
-        a.geom = window_of(c, br);
+        a.geom = geo;
         a.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d_k);
         a.scale = 1.f / sqrtf((float)c.d_k);
         a.gates = gates;

@@ -129,6 +129,9 @@ struct BwdFinalizeArgs {
     double inv_freq[64];
 };
 cudaError_t launch_bwd_finalize(const BwdFinalizeArgs &a, bool bf16, cudaStream_t s);
+// rowdot = dout . o per row (o fp32 [B, L, H, d]), written in [B, L, H] and [B, H, L] order
+cudaError_t launch_rowdot(const void *dout, const float *o, long long rows, int d, int L, int H, bool bf16,
+                          float *rowdot, float *rowdot_hm, cudaStream_t s);
 // dgates[h*3 + col] = sum over (b, t) of rowdot[(b*L + t)*H + h]
 cudaError_t launch_gate_grad(const float *rowdot, int B, int L, int H, int col, float *dgates, cudaStream_t s);
 

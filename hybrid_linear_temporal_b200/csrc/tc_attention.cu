@@ -78,6 +78,7 @@ struct TcAttnParams {
     float *acc;
     const float *acc2;  // optional second accumulator, added in the final modes
     __nv_bfloat16 *out;
+    float *lse_out;  // optional [B, H, L]: log2-domain log-sum-exp of each row's scaled scores
     int *dev_err;
 };
 
@@ -424,6 +425,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const int tok = seg_f * p.Pseg + s0 + j * kBM + row;
             const size_t base = (((size_t)b * p.L + tok) * p.H + h) * kD;
             const float scale = p.gates[h * 3 + p.gate_col] / l_run;
+            if (p.lse_out && row < nqj) p.lse_out[((size_t)b * p.H + h) * p.L + tok] = m_ref + log2f(l_run);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t r[32];
@@ -503,7 +505,7 @@ public:
 
     cudaError_t run(const void *q, const void *k, const void *v, int L, WindowGeom g, const float *gates,
                     int gate_col, int mode, float *acc, const float *acc2, void *out, int *dev_err,
-                    cudaStream_t s, bool *done) override {
+                    cudaStream_t s, bool *done, float *lse_out) override {
         *done = false;
         int Pseg, Fseg;
         if (!geometry(L, g, &Pseg, &Fseg)) return cudaSuccess;
@@ -530,6 +532,7 @@ public:
         p.acc2 = acc2;
         p.out = static_cast<__nv_bfloat16 *>(out);
         p.dev_err = dev_err;
+        p.lse_out = lse_out;
         const size_t smem = sizeof(Smem) + 1024;
         if (!attr_set_) {
             cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

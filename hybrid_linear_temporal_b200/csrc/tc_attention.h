@@ -16,9 +16,11 @@ public:
     // Sets *done = false (and enqueues nothing) when this case is not covered,
     // so the caller runs the CUDA-core kernel instead.
     // acc2 (may be null) is a second fp32 accumulator added in the final modes.
+    // lse_out (may be null) receives each row's log2-domain log-sum-exp, [B, H, L].
     virtual cudaError_t run(const void *q, const void *k, const void *v, int L, WindowGeom g,
                             const float *gates, int gate_col, int mode, float *acc, const float *acc2,
-                            void *out, int *dev_err, cudaStream_t s, bool *done) = 0;
+                            void *out, int *dev_err, cudaStream_t s, bool *done,
+                            float *lse_out = nullptr) = 0;
     // True when run() would take this case (rather than leave it to the CUDA-core kernel).
     virtual bool covers(int L, WindowGeom g) const = 0;
 };

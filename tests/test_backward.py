@@ -3,9 +3,12 @@ the oracle's reverse-mode derivatives on the same seeded inputs.
 
 Tolerances: gradients returned in bf16 (dq, dk, dv of a bf16 layer) -- relative
 L2 <= 5e-3 and max-abs <= 2e-2 * max(1, max |ref|) (one bf16 rounding of each
-element on top of fp32 arithmetic); gradients returned in fp32 (dalpha, dbeta,
-dgates, dS0, and everything of an fp32 layer) -- relative L2 <= 1e-3 for bf16
-layers (fp32 arithmetic from bf16 inputs) and 1e-4 for fp32 layers.
+element on top of the arithmetic); gradients returned in fp32 (dalpha, dbeta,
+dS0, and everything of an fp32 layer) -- relative L2 <= 1e-3 for bf16 layers
+(fp32 arithmetic from bf16 inputs) and 1e-4 for fp32 layers.  dgates = dout . o
+takes the branch outputs of the forward, whose bf16 tensor-core path rounds the
+softmax weights to bf16, so for bf16 layers it carries the forward's relative
+L2 bound of 5e-3.
 """
 import numpy as np
 import pytest
@@ -34,13 +37,13 @@ def _dout(wl, seed):
     return bf16_bits(x) if wl.dtype == "bf16" else x.astype(np.float32)
 
 
-def _check(got, ref, what, returned_bf16, layer_bf16):
+def _check(got, ref, what, returned_bf16, layer_bf16, tol_bf16_layer=1e-3):
     e = errors(got, ref)
     if returned_bf16:
         lim = 2e-2 * max(1.0, float(np.abs(ref).max()))
         assert e["rel_l2"] <= 5e-3 and e["max_abs"] <= lim, f"{what}: {e}"
     else:
-        tol = 1e-3 if layer_bf16 else 1e-4
+        tol = tol_bf16_layer if layer_bf16 else 1e-4
         assert e["rel_l2"] <= tol, f"{what}: {e} vs {tol}"
     return e
 
@@ -73,7 +76,7 @@ def backward_compare(torch, wl, seed=0, branches=BRANCHES, S0=False, dS_final=Fa
         res[n] = _check(to_numpy64(got[n]), ref[n], f"{wl.name} {n}", bf, bf)
     cols = [i for i, n in enumerate(BRANCHES) if n in branches]
     res["dgates"] = _check(to_numpy64(got["dgates"])[:, cols], ref["dgates"][:, cols], f"{wl.name} dgates",
-                           False, bf)
+                           False, bf, tol_bf16_layer=5e-3)
     assert np.abs(to_numpy64(got["dgates"])[:, [i for i in range(3) if i not in cols]]).max(initial=0) == 0
     if "gdn" in branches:
         for n in ("dalpha", "dbeta", "dS0"):
@@ -140,3 +143,10 @@ def test_backward_rejects_printed_update_form(torch_cuda):
     # the attention branches alone are fine with either update form
     layer.backward(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], dev["gates"], dout, branches=3)
     layer.close()
+
+
+def test_backward_rollout_shaped_bf16(torch_cuda):
+    """Frames of the 480P rollout (1560 tokens, windows 1560), fewer frames and
+    heads so that the oracle runs in seconds; both branches on the tensor cores."""
+    wl = WORKLOADS["rollout_480p"].with_(H=2, L=1560 * 5, dilation=2)
+    backward_compare(torch_cuda, wl, S0=True, dS_final=True)
