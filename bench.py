@@ -48,6 +48,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-logits measurement")
     return ap.parse_args()
 
 
@@ -482,6 +483,34 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.nbytes),
                "ms_per_step": round(ms_e2e, 3), "steps": n_e2e}
 
+    # FP8 logits variant (Q K^T in e4m3): the same step and the attention launches alone
+    fp8 = None
+    if not args.no_fp8:
+        l8 = HLTA.for_workload(wl, attn_fp8=1)
+
+        def step8():
+            l8.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["gates"], out=out, stream=stream)
+        for _ in range(3):
+            step8()
+        torch.cuda.synchronize()
+        n8 = max(3, min(args.steps, 10))
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(n8):
+            step8()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        ms8 = max_over_ranks(g0.elapsed_time(g1) / n8, world)
+        iso8 = attention_alone(l8, d, out, stream)
+        fp8 = {"ms_per_step": round(ms8, 4), "value": round(world * wl.B * wl.L / (ms8 * 1e-3), 1),
+               "unit": "tokens/s", "steps": n8,
+               "dtype": "Q K^T e4m3 (one scale per 128-row tile), P V bf16"}
+        if iso8:
+            r8 = attention_roofline(iso8[0], iso8[1], wl, peaks, sustained=False)
+            fp8["attention_alone"] = {"ms_swa": round(iso8[0], 4), "ms_dswa": round(iso8[1], 4),
+                                      "achieved_tflops": r8["achieved"]}
+        l8.close()
+
     bwd = None
     if not args.no_backward:
         bwd = backward_measure(layer, d, wl, stream, max(1, min(args.steps, 3)), world)
@@ -501,7 +530,7 @@ def run_ours(args, world, rank, local):
                 "branches": branches,
                 "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(prof.get("kernel_launches", 0)),
-                "clocks": clk, "backward": bwd}
+                "clocks": clk, "backward": bwd, "fp8": fp8}
         print(json.dumps(line), flush=True)
     layer.close()
 

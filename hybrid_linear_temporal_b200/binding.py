@@ -29,7 +29,7 @@ class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "B", "H", "d_k", "d_v", "tokens_per_frame", "swa_window", "dswa_window",
         "dswa_dilation", "chunk", "dtype", "max_seq_len", "max_stream_tokens", "gdn_form",
-        "window_mode")] + [("rope_base", ctypes.c_float)]
+        "window_mode")] + [("rope_base", ctypes.c_float), ("attn_fp8", ctypes.c_int)]
 
 
 class ProfileData(ctypes.Structure):
@@ -129,11 +129,11 @@ class HLTA:
 
     def __init__(self, B, H, d_k, d_v, tokens_per_frame, swa_window, dswa_window, dilation,
                  chunk=64, dtype="bf16", max_seq_len=1, max_stream_tokens=0, gdn_form=0,
-                 window_mode=0, rope_base=0.0):
+                 window_mode=0, rope_base=0.0, attn_fp8=0):
         self.lib = load_library()
         self.cfg = Config(B, H, d_k, d_v, tokens_per_frame, swa_window, dswa_window, dilation,
                           chunk, BF16 if dtype == "bf16" else FP32, max_seq_len, max_stream_tokens,
-                          gdn_form, window_mode, rope_base)
+                          gdn_form, window_mode, rope_base, attn_fp8)
         self.dtype = dtype
         h = ctypes.c_void_p()
         _check(self.lib, self.lib.hlta_create(ctypes.byref(self.cfg), ctypes.byref(h)))
@@ -141,10 +141,10 @@ class HLTA:
 
     @classmethod
     def for_workload(cls, wl, max_seq_len=None, max_stream_tokens=0, gdn_form=0, window_mode=0,
-                     rope_base=0.0):
+                     rope_base=0.0, attn_fp8=0):
         return cls(wl.B, wl.H, wl.d_k, wl.d_v, wl.P, wl.swa_window, wl.dswa_window, wl.dilation,
                    wl.chunk, wl.dtype, max_seq_len or wl.L, max_stream_tokens, gdn_form, window_mode,
-                   rope_base)
+                   rope_base, attn_fp8)
 
     def close(self):
         if getattr(self, "h", None):

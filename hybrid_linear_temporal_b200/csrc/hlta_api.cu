@@ -94,6 +94,8 @@ struct hlta_handle {
     float *acc2 = nullptr;
     // rotated q and k for the attention branches (rope_base > 0)
     void *q_rot = nullptr, *k_rot = nullptr;
+    // e4m3 copies of q and k and their tile scales (attn_fp8)
+    hlta::Fp8Scratch f8 = {nullptr, nullptr, nullptr, nullptr};
     // backward scratch: one block allocated at the first hlta_backward, kept
     char *bw_block = nullptr;
     float *g_dq = nullptr, *g_dk = nullptr, *g_dv = nullptr, *g_dq_att = nullptr, *g_dk_att = nullptr;
@@ -157,6 +159,9 @@ hlta_status check_config(const hlta_config *c) {
         return fail(HLTA_ERR_UNSUPPORTED, "centred windows need the whole sequence: not with streaming");
     if (c->rope_base > 0.f && c->window_mode != HLTA_WINDOW_CENTRED)
         return fail(HLTA_ERR_UNSUPPORTED, "rotary embedding is provided with centred windows");
+    if (c->attn_fp8 != 0 && c->attn_fp8 != 1) return fail(HLTA_ERR_INVALID_ARG, "attn_fp8 must be 0 or 1");
+    if (c->attn_fp8 && (c->dtype != HLTA_BF16 || c->d_k != 128 || c->d_v != 128))
+        return fail(HLTA_ERR_UNSUPPORTED, "attn_fp8 needs dtype HLTA_BF16 and d_k = d_v = 128");
     if ((c->d_k != 64 && c->d_k != 128) || (c->d_v != 64 && c->d_v != 128))
         return fail(HLTA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128");
     if (c->chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64");
@@ -313,7 +318,8 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
             bool done = false;
             const int mode = last ? (idx == 0 ? hlta::OUT_FINAL_ONLY : hlta::OUT_FINAL) : hlta::OUT_STORE;
             cudaError_t e = h->tc_attn->run(att.q, kst, vst, nq, geo[br], in.gates, br, mode, h->acc,
-                                            last ? h->acc2 : nullptr, out, h->dev_err, s, &done);
+                                            last ? h->acc2 : nullptr, out, h->dev_err, s, &done, nullptr,
+                                            c.attn_fp8 ? &h->f8 : nullptr);
             if (e != cudaSuccess || !done)
                 return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
             ps.done(1);
@@ -331,7 +337,8 @@ hlta_status run_pass(hlta_handle *h, const Inputs &in, long long pos0, int nq, c
             bool done = false;
             if (one_shot && h->tc_attn) {
                 cudaError_t e = h->tc_attn->run(att.q, kst, vst, nq, g, in.gates, br, mode, h->acc,
-                                                nullptr, out, h->dev_err, s, &done);
+                                                nullptr, out, h->dev_err, s, &done, nullptr,
+                                                c.attn_fp8 ? &h->f8 : nullptr);
                 if (e != cudaSuccess)
                     return fail(HLTA_ERR_CUDA, "tensor-core attention: %s", cudaGetErrorString(e));
             }
@@ -431,6 +438,12 @@ hlta_status hlta_create(const hlta_config *cfg, hlta_handle **out) {
     };
     const size_t acc_bytes = (size_t)cfg->B * h->acc_rows * cfg->H * cfg->d_v * sizeof(float);
     bool okk = alloc((void **)&h->acc, acc_bytes) && alloc((void **)&h->dev_err, sizeof(int));
+    if (okk && cfg->attn_fp8) {
+        const size_t n8 = (size_t)cfg->B * cfg->max_seq_len * cfg->H * 128;
+        const size_t ns = hlta::fp8_scale_floats(cfg->B, cfg->H, cfg->max_seq_len, cfg->tokens_per_frame);
+        okk = alloc(&h->f8.q8, n8) && alloc(&h->f8.k8, n8) && alloc((void **)&h->f8.sq, ns * sizeof(float)) &&
+              alloc((void **)&h->f8.sk, ns * sizeof(float));
+    }
     if (okk && cfg->rope_base > 0.f) {
         const size_t qk_bytes = (size_t)cfg->B * cfg->max_seq_len * cfg->H * cfg->d_k * h->elem_bytes;
         okk = alloc(&h->q_rot, qk_bytes) && alloc(&h->k_rot, qk_bytes);
@@ -489,6 +502,10 @@ hlta_status hlta_destroy(hlta_handle *h) {
     cudaFree(h->q_rot);
     cudaFree(h->k_rot);
     cudaFree(h->bw_block);
+    cudaFree(h->f8.q8);
+    cudaFree(h->f8.k8);
+    cudaFree(h->f8.sq);
+    cudaFree(h->f8.sk);
     if (h->side) cudaStreamDestroy(h->side);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);

@@ -38,6 +38,7 @@
 // band it misses, and tiles crossing a band edge or a segment end are masked
 // per element.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdio.h>
 
 #include "common.cuh"
@@ -66,6 +67,7 @@ struct KeyTile {
     int s0;      // first key row inside the segment
     int rbase;   // rearranged position of that row
     int kvalid;  // rows of this tile inside the segment
+    float sk;    // FP8 variant: the e4m3 scale of this k tile (1 otherwise)
     uint8_t use[kQT], full[kQT];
 };
 
@@ -79,6 +81,9 @@ struct TcAttnParams {
     const float *acc2;  // optional second accumulator, added in the final modes
     __nv_bfloat16 *out;
     float *lse_out;  // optional [B, H, L]: log2-domain log-sum-exp of each row's scaled scores
+    // FP8 variant: per-tile scales of the e4m3 q and k, [B*Fseg][H][nblk] (128-row blocks)
+    const float *sq, *sk;
+    int nblk;
     int *dev_err;
 };
 
@@ -153,9 +158,14 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
+// kF8: q and k arrive as e4m3 tiles (128 one-byte columns, one TMA box) with a
+// scale per 128-row tile; Q K^T runs as kind::f8f6f4 and the two tiles' scales
+// multiply the softmax exponent.  P V stays bf16.
+template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const TcAttnParams p) {
+    constexpr uint32_t kQKBytes = kF8 ? kTileBytes / 2 : kTileBytes;  // one Q or K tile
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,6 +196,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 k.s0 = t * kBN;
                 k.rbase = base + t * kBN;
                 k.kvalid = min(kBN, p.Pseg - t * kBN);
+                k.sk = kF8 ? p.sk[((size_t)k.seg * p.H + h) * p.nblk + t] : 1.f;
 #pragma unroll
                 for (int j = 0; j < kQT; ++j) {
                     const int lo = r_min + j * kBM, hi = lo + nqs[j] - 1;
@@ -226,10 +237,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
             const int qseg = b * p.Fseg + seg_f;
-            mbar_expect_tx(&sm.bar_q, nq1 > 0 ? 2 * kTileBytes : kTileBytes);
+            mbar_expect_tx(&sm.bar_q, nq1 > 0 ? 2 * kQKBytes : kQKBytes);
             for (int j = 0; j < (nq1 > 0 ? 2 : 1); ++j) {
                 tma_load_4d(sm.q[j], &tmQ, 0, h, s0 + j * kBM, qseg, &sm.bar_q);
-                tma_load_4d(sm.q[j] + kHalfBytes, &tmQ, 64, h, s0 + j * kBM, qseg, &sm.bar_q);
+                if (!kF8) tma_load_4d(sm.q[j] + kHalfBytes, &tmQ, 64, h, s0 + j * kBM, qseg, &sm.bar_q);
             }
             int issued = 0;
             for (int u = 0; u < 2 * nkt; ++u) {
@@ -237,9 +248,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (u >= kSlots && !mbar_wait(&sm.empty[slot], ((u / kSlots) - 1) & 1, abort, p.dev_err)) break;
                 const KeyTile &kt = sm.kt[u >> 1];
                 const CUtensorMap *map = (u & 1) ? &tmV : &tmK;
-                mbar_expect_tx(&sm.full[slot], kTileBytes);
+                const bool one_box = kF8 && !(u & 1);
+                mbar_expect_tx(&sm.full[slot], one_box ? kQKBytes : kTileBytes);
                 tma_load_4d(sm.kv[slot], map, 0, h, kt.s0, kt.seg, &sm.full[slot]);
-                tma_load_4d(sm.kv[slot] + kHalfBytes, map, 64, h, kt.s0, kt.seg, &sm.full[slot]);
+                if (!one_box) tma_load_4d(sm.kv[slot] + kHalfBytes, map, 64, h, kt.s0, kt.seg, &sm.full[slot]);
                 issued = u + 1;
             }
             if (*abort) {
@@ -256,7 +268,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // Per key tile t: PV0(t), QK0(t+1), PV1(t), QK1(t+1).  QK_j(t+1) reuses
         // S_j's columns, which hold P_j(t): it is issued after PV_j(t).
         if (lane == 0) {
-            const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+            const uint32_t idesc_qk = kF8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
             int npv[kQT] = {0, 0};
             bool live = !*abort && mbar_wait(&sm.bar_q, 0, abort, p.dev_err);
@@ -264,11 +276,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             auto issue_qk = [&](int j, uint32_t ka) {
                 tc_fence_after();
                 const uint32_t qa = smem_u32(sm.q[j]);
+                if constexpr (kF8) {
+                    // 128 one-byte columns per row: four K = 32 steps within one swizzle atom
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
-                    umma_ss(tmem + j * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                            idesc_qk, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kD / 32; ++kk)
+                        umma_ss_f8(tmem + j * 128, smem_desc_sw128(qa + kk * 32, 16, 1024),
+                                   smem_desc_sw128(ka + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint32_t off = (kk < 4) ? kk * 32 : kHalfBytes + (kk - 4) * 32;
+                        umma_ss(tmem + j * 128, smem_desc_sw128(qa + off, 16, 1024),
+                                smem_desc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    }
                 }
                 umma_commit(&sm.bar_s[j]);
             };
@@ -335,7 +355,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint32_t colS = j * 128, colO = 256 + j * 128;
         const int nqj = j == 0 ? nq0 : nq1;
         const int r_q = r_min + j * kBM + row;
-        const float sl2 = p.scale_log2;
+        const float sq = (kF8 && nqj > 0) ? p.sq[((size_t)(b * p.Fseg + seg_f) * p.H + h) * p.nblk + (s0 + j * kBM) / kBM]
+                                          : 1.f;
         float m_ref = -INFINITY, l_run = 0.f;
         int n = 0;
         bool ok = !*abort;
@@ -344,6 +365,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (!ktr.use[j]) continue;
             const bool full = ktr.full[j];
             const int rbase = ktr.rbase, kvalid = ktr.kvalid;
+            // logits scale: log2(e)/sqrt(d), times the e4m3 tiles' scales
+            const float sl2 = kF8 ? p.scale_log2 * sq * ktr.sk : p.scale_log2;
             // waits are made warp-uniform: the TMEM loads below are warp-collective
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_s[j], n & 1, abort, p.dev_err))) {
                 ok = false;
@@ -444,6 +467,57 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
 }
 
+// e4m3 quantization of q or k for the FP8 Q K^T path: one CTA per (128-row
+// block, head, segment), one thread per row.  scale = max |x| / 448 over the
+// 128 x 128 tile (448: the largest finite e4m3 value); x8 = e4m3(x / scale),
+// rounded to nearest and saturating.  Rows past the segment end are not
+// written (the kernel's tensor map never reads them).
+__global__ void __launch_bounds__(128) quant_e4m3_kernel(const __nv_bfloat16 *x, uint8_t *x8, float *scales,
+                                                         int Pseg, int H, int nblk) {
+    const int blk = blockIdx.x, h = blockIdx.y, seg = blockIdx.z;
+    const int r = blk * kBM + threadIdx.x;
+    const bool live = r < Pseg;
+    const size_t row = ((size_t)seg * Pseg + (live ? r : 0)) * H + h;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + row * kD);
+    float v[kD];
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < kD / 8; ++c) {
+        uint4 u = live ? src[c] : make_uint4(0, 0, 0, 0);
+        const __nv_bfloat162 *pr = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            v[8 * c + 2 * e] = __low2float(pr[e]);
+            v[8 * c + 2 * e + 1] = __high2float(pr[e]);
+            amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * e]), fabsf(v[8 * c + 2 * e + 1])));
+        }
+    }
+    __shared__ float wmax[4];
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    const float scale = amax > 0.f ? amax / 448.f : 1.f;
+    const float inv = 1.f / scale;
+    if (threadIdx.x == 0) scales[((size_t)seg * H + h) * nblk + blk] = scale;
+    if (!live) return;
+    uint4 *dst = reinterpret_cast<uint4 *>(x8 + row * kD);
+#pragma unroll
+    for (int c = 0; c < kD / 16; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = 16 * c + 4 * e;
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[i] * inv, v[i + 1] * inv), __NV_SATFINITE,
+                                                         __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v[i + 2] * inv, v[i + 3] * inv),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            w[e] = lo | (hi << 16);
+        }
+        dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
@@ -471,6 +545,20 @@ bool make_map(CUtensorMap *map, const void *base, int H, int Pseg, int segs) {
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBN, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D view (d, H, Pseg, B*Fseg) of a [B, L, H, d] e4m3 tensor, box (128, 1, 128, 1):
+// one 128-byte swizzle atom per row.
+bool make_map8(CUtensorMap *map, const void *base, int H, int Pseg, int segs) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)Pseg, (cuuint64_t)segs};
+    const cuuint64_t strides[3] = {(cuuint64_t)kD, (cuuint64_t)H * kD, (cuuint64_t)Pseg * H * kD};
+    const cuuint32_t box[4] = {(cuuint32_t)kD, 1, (cuuint32_t)kBN, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -505,14 +593,25 @@ public:
 
     cudaError_t run(const void *q, const void *k, const void *v, int L, WindowGeom g, const float *gates,
                     int gate_col, int mode, float *acc, const float *acc2, void *out, int *dev_err,
-                    cudaStream_t s, bool *done, float *lse_out) override {
+                    cudaStream_t s, bool *done, float *lse_out, const Fp8Scratch *f8) override {
         *done = false;
         int Pseg, Fseg;
         if (!geometry(L, g, &Pseg, &Fseg)) return cudaSuccess;
 
         CUtensorMap mq, mk, mv;
         const int segs = cfg_.B * Fseg;
-        if (!make_map(&mq, q, cfg_.H, Pseg, segs) || !make_map(&mk, k, cfg_.H, Pseg, segs) ||
+        const int nblk = (Pseg + kBM - 1) / kBM;
+        if (f8) {
+            const dim3 qgrid(nblk, cfg_.H, segs);
+            quant_e4m3_kernel<<<qgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16 *>(q),
+                                                   static_cast<uint8_t *>(f8->q8), f8->sq, Pseg, cfg_.H, nblk);
+            quant_e4m3_kernel<<<qgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16 *>(k),
+                                                   static_cast<uint8_t *>(f8->k8), f8->sk, Pseg, cfg_.H, nblk);
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        if (!(f8 ? make_map8(&mq, f8->q8, cfg_.H, Pseg, segs) && make_map8(&mk, f8->k8, cfg_.H, Pseg, segs)
+                 : make_map(&mq, q, cfg_.H, Pseg, segs) && make_map(&mk, k, cfg_.H, Pseg, segs)) ||
             !make_map(&mv, v, cfg_.H, Pseg, segs))
             return cudaErrorInvalidValue;
         TcAttnParams p;
@@ -533,15 +632,24 @@ public:
         p.out = static_cast<__nv_bfloat16 *>(out);
         p.dev_err = dev_err;
         p.lse_out = lse_out;
+        p.sq = f8 ? f8->sq : nullptr;
+        p.sk = f8 ? f8->sk : nullptr;
+        p.nblk = nblk;
         const size_t smem = sizeof(Smem) + 1024;
         if (!attr_set_) {
-            cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)smem);
+            cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
             if (e != cudaSuccess) return e;
             attr_set_ = true;
         }
         const dim3 grid(Fseg * p.qblocks_per_seg, cfg_.H, cfg_.B);
-        attn_tc_kernel<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
+        if (f8)
+            attn_tc_kernel<true><<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
+        else
+            attn_tc_kernel<false><<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
         *done = true;
         return cudaGetLastError();
     }
@@ -552,6 +660,13 @@ private:
 };
 
 }  // namespace
+
+size_t fp8_scale_floats(int B, int H, int max_len, int tokens_per_frame) {
+    const size_t swa = (size_t)(max_len + kBM - 1) / kBM;
+    const size_t frames = (size_t)max_len / tokens_per_frame + 1;
+    const size_t dswa = frames * (size_t)((tokens_per_frame + kBM - 1) / kBM);
+    return (size_t)B * H * (swa > dswa ? swa : dswa);
+}
 
 TcAttention *TcAttention::create(const hlta_config &cfg, long long) {
     if (cfg.dtype != HLTA_BF16 || cfg.d_k != kD || cfg.d_v != kD) return nullptr;

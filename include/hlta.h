@@ -113,6 +113,12 @@ typedef struct {
                               RoPE for these blocks; reading: channel pair (2m, 2m+1) of the
                               token at position t turns by t * rope_base^(-2m/d_k)); 0: none.
                               Centred windows only.  The memory branch never rotates. */
+    int attn_fp8;          /* 1: the SWA/DSWA logits Q K^T run in FP8 (e4m3, one scale per
+                              128-row tile of q and of k, the pages' FP8 attention
+                              quantization) on the tensor cores; P V stays bf16.  Needs
+                              dtype HLTA_BF16 and d_k = d_v = 128; applies where the
+                              tensor-core kernel takes the branch (full frames), elsewhere
+                              the branch runs unquantized.  hlta_backward does not use it. */
 } hlta_config;
 
 typedef struct hlta_handle hlta_handle;

@@ -38,7 +38,7 @@ def test_version(lib):
 def _cfg(**kw):
     base = dict(B=1, H=2, d_k=64, d_v=64, tokens_per_frame=4, swa_window=8, dswa_window=8,
                 dswa_dilation=2, chunk=64, dtype=binding.BF16, max_seq_len=128, max_stream_tokens=0,
-                gdn_form=binding.GDN_DECAYED, window_mode=binding.WINDOW_CAUSAL, rope_base=0.0)
+                gdn_form=binding.GDN_DECAYED, window_mode=binding.WINDOW_CAUSAL, rope_base=0.0, attn_fp8=0)
     base.update(kw)
     return binding.Config(*[base[n] for n, _ in binding.Config._fields_])
 
@@ -69,6 +69,10 @@ def test_create_rejects_bad_config_before_device(lib, field, value, status):
     (dict(window_mode=binding.WINDOW_CAUSAL, rope_base=10000.0), binding.ERR_UNSUPPORTED),
     # a centred window reaches keys after the query: not available token by token
     (dict(window_mode=binding.WINDOW_CENTRED, max_stream_tokens=16), binding.ERR_UNSUPPORTED),
+    (dict(attn_fp8=2), binding.ERR_INVALID_ARG),
+    # the FP8 logits path exists for the bf16 tensor-core kernel (d = 128) only
+    (dict(attn_fp8=1), binding.ERR_UNSUPPORTED),
+    (dict(attn_fp8=1, dtype=binding.FP32, d_k=128, d_v=128), binding.ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_window_config(lib, over, status):
     h = ctypes.c_void_p()

@@ -334,3 +334,46 @@ def test_rejects_bad_tensors(torch_cuda):
     with pytest.raises(ValueError):
         layer.forward(dev["q"].float(), dev["k"], dev["v"], dev["alpha"], dev["beta"], dev["gates"])
     layer.close()
+
+
+# FP8 logits: Q K^T in e4m3 with one scale per 128-row tile, P V in bf16.  The
+# bound is the specification's looser FP8 tolerance, derived from a CPU model of
+# the e4m3 rounding (relative L2 3e-4 at unit query scale, 4.5e-3 at 16x on the
+# 4k clip) plus the bf16 path's own error: relative L2 <= 1.5e-2, max-abs <= 5e-2.
+FP8_TOL = {"rel_l2": 1.5e-2, "max_abs": 5e-2}
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 16.0])
+def test_fp8_logits_clip_4k(torch_cuda, q_scale):
+    wl = WORKLOADS["clip_4k"]
+    inp = make_inputs(wl, q_scale=q_scale)
+    dev = to_device(inp)
+    g = inp.gates.astype(np.float64)
+    l8, l16 = layer_for(wl, attn_fp8=1), layer_for(wl)
+    for i, (name, dil, w) in enumerate((("swa", 1, wl.swa_window), ("dswa", wl.dilation, wl.dswa_window))):
+        ref = g[None, None, :, i, None] * oracle.attention(name, inp.q, inp.k, inp.v, wl.P, dil, w)
+        o8 = to_numpy64(run_gpu(l8, dev, branches=1 << i)[0])
+        o16 = to_numpy64(run_gpu(l16, dev, branches=1 << i)[0])
+        e = errors(o8, ref)
+        assert e["rel_l2"] <= FP8_TOL["rel_l2"] and e["max_abs"] <= FP8_TOL["max_abs"], f"{name} fp8: {e}"
+        if q_scale > 1:
+            # the e4m3 path ran: it differs from the bf16 path by about the modelled rounding
+            assert errors(o8, o16)["rel_l2"] > 5e-4, name
+    # the whole layer (memory branch unchanged)
+    if q_scale == 1.0:
+        ref = oracle.forward(inp)["out"]
+        e = errors(to_numpy64(run_gpu(l8, dev)[0]), ref)
+        assert e["rel_l2"] <= FP8_TOL["rel_l2"] and e["max_abs"] <= FP8_TOL["max_abs"], f"layer fp8: {e}"
+    l8.close()
+    l16.close()
+
+
+def test_fp8_logits_ragged_frames_fall_back(torch_cuda):
+    """DSWA frames of 50 tokens (no tensor-core tiles) run unquantized; SWA in e4m3."""
+    wl = WORKLOADS["clip_4k"].with_(H=2, L=1000, P=50, swa_window=300, dswa_window=120, dilation=3)
+    inp = make_inputs(wl)
+    l8 = layer_for(wl, attn_fp8=1)
+    out, _ = run_gpu(l8, to_device(inp))
+    e = errors(to_numpy64(out), oracle.forward(inp)["out"])
+    assert e["rel_l2"] <= FP8_TOL["rel_l2"] and e["max_abs"] <= FP8_TOL["max_abs"], e
+    l8.close()
