@@ -11,9 +11,9 @@
 // recurrence's reverse mode) runs in four kernels:
 //   gdn_bwd_prep   per chunk: T, W, T diag(beta) V, diag(D) K, and
 //                  Lc = dO^T (diag(gamma) Q - P W)
-//   gdn_bwd_fscan  per (b, h, 16 state rows), chunks in order: the chunk start
+//   gdn_bwd_fscan  per (b, h, 32 state rows), chunks in order: the chunk start
 //                  states S0 and U (rows of S evolve independently)
-//   gdn_bwd_dscan  per (b, h, 16 rows), chunks in reverse: the gradient of each
+//   gdn_bwd_dscan  per (b, h, 32 rows), chunks in reverse: the gradient of each
 //                  chunk's end state, dS <- gamma_C dS - (dS (DK)^T) W + Lc
 //   gdn_bwd_local  per chunk: dq, dk, dv, dalpha, dbeta and dout . o
 // All arithmetic is fp32; matrix products use a shared-memory-tiled block GEMM.
@@ -207,72 +207,134 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_prep(GdnBwdArgs a) {
     }
 }
 
+// Asynchronous 16-byte global -> shared copies (completion by commit groups).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// n floats (a multiple of 4, 16-byte aligned at both ends) by the whole block
+__device__ __forceinline__ void copy_async(float *dst, const float *src, int n) {
+    for (int i = threadIdx.x * 4; i < n; i += kThreads * 4) cp_async16(dst + i, src + i);
+}
+
+constexpr int kScanRows = 32;  // state rows per scan CTA
+
+template <int DK, int DV>
+constexpr size_t fscan_smem_floats() {
+    return 2 * (2 * (size_t)kC * DK + (size_t)kC * kScanRows + 4) + (size_t)kScanRows * DK + kC * kScanRows +
+           kKT * (kScanRows + DK);
+}
+template <int DK, int DV>
+constexpr size_t dscan_smem_floats() {
+    return 2 * (2 * (size_t)kC * DK + (size_t)kScanRows * DK + 4) + (size_t)kScanRows * DK + kScanRows * kC +
+           kKT * (kScanRows + DK);
+}
+
 // ---------------------------------------------------------------------------
-// gdn_bwd_fscan: chunk start states and U, 16 rows of S per CTA.
+// gdn_bwd_fscan: chunk start states and U, 32 rows of S per CTA.  The next
+// chunk's W, diag(D) K, the row slice of T diag(beta) V and l_C are copied into
+// shared memory (double buffer) while the current chunk is computed.
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads) gdn_bwd_fscan(GdnBwdArgs a) {
-    constexpr int R = 16;
-    __shared__ float Sr[R][DK];
-    __shared__ float Ub[kC][R];
-    __shared__ float stage[kKT * (kC + DK)];
+    constexpr int R = kScanRows;
+    extern __shared__ __align__(16) float fsm[];
+    float *buf[2];
+    buf[0] = fsm;
+    buf[1] = fsm + (2 * kC * DK + kC * R + 4);
+    float *Sr = fsm + 2 * (2 * kC * DK + kC * R + 4);
+    float *Ub = Sr + R * DK;
+    float *stage = Ub + kC * R;
     const int r0 = blockIdx.x * R, bh = blockIdx.y;
     const int nc = (a.L + kC - 1) / kC;
     const int tid = threadIdx.x;
+    // buffer layout: W [kC][DK], Kd [kC][DK], TbV rows slice [kC][R], l (4 floats, the last is l_C)
+    auto prefetch = [&](int ci, float *bf) {
+        const size_t cidx = (size_t)bh * nc + ci;
+        copy_async(bf, a.bw_W + cidx * kC * DK, kC * DK);
+        copy_async(bf + kC * DK, a.bw_Kd + cidx * kC * DK, kC * DK);
+        const float *TbV = a.bw_TbV + cidx * kC * DV + r0;
+        for (int i = tid; i < kC * (R / 4); i += kThreads)
+            cp_async16(bf + 2 * kC * DK + (i / (R / 4)) * R + (i % (R / 4)) * 4, TbV + (i / (R / 4)) * DV + (i % (R / 4)) * 4);
+        if (tid == 0) cp_async16(bf + 2 * kC * DK + kC * R, a.bw_ell + cidx * kC + kC - 4);
+    };
     for (int idx = tid; idx < R * DK; idx += kThreads)
-        Sr[idx / DK][idx % DK] = a.S0 ? a.S0[((size_t)bh * DV + r0 + idx / DK) * DK + idx % DK] : 0.f;
-    __syncthreads();
+        Sr[idx] = a.S0 ? a.S0[((size_t)bh * DV + r0 + idx / DK) * DK + idx % DK] : 0.f;
+    prefetch(0, buf[0]);
+    cp_async_commit();
     for (int ci = 0; ci < nc; ++ci) {
+        if (ci + 1 < nc) prefetch(ci + 1, buf[(ci + 1) & 1]);
+        cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        const float *bf = buf[ci & 1];
         const size_t cidx = (size_t)bh * nc + ci;
         float *Sg = a.bw_S + cidx * DV * DK + (size_t)r0 * DK;
-        for (int idx = tid; idx < R * DK; idx += kThreads) Sg[idx] = Sr[idx / DK][idx % DK];
+        for (int idx = tid; idx < R * DK; idx += kThreads) Sg[idx] = Sr[idx];
         // U[:, rows] = T diag(beta) V[:, rows] - W S_rows^T
-        const float *TbV = a.bw_TbV + cidx * kC * DV;
-        for (int idx = tid; idx < kC * R; idx += kThreads) Ub[idx / R][idx % R] = TbV[(idx / R) * DV + r0 + idx % R];
-        block_gemm<kC, R>(mat(a.bw_W + cidx * kC * DK, DK, 1), mat(&Sr[0][0], 1, DK), DK, &Ub[0][0], R, 1, -1.f,
-                          1.f, stage);
+        for (int idx = tid; idx < kC * R; idx += kThreads) Ub[idx] = bf[2 * kC * DK + idx];
+        block_gemm<kC, R>(mat(bf, DK, 1), mat(Sr, 1, DK), DK, Ub, R, 1, -1.f, 1.f, stage);
         float *Ug = a.bw_U + cidx * kC * DV;
-        for (int idx = tid; idx < kC * R; idx += kThreads) Ug[(idx / R) * DV + r0 + idx % R] = Ub[idx / R][idx % R];
+        for (int idx = tid; idx < kC * R; idx += kThreads) Ug[(idx / R) * DV + r0 + idx % R] = Ub[idx];
         // S_rows <- gamma_C S_rows + U[:, rows]^T diag(D) K
-        const float gC = expf(a.bw_ell[cidx * kC + kC - 1]);
-        block_gemm<R, DK>(mat(&Ub[0][0], 1, R), mat(a.bw_Kd + cidx * kC * DK, DK, 1), kC, &Sr[0][0], DK, 1, 1.f, gC,
-                          stage);
+        const float gC = expf(bf[2 * kC * DK + kC * R + 3]);
+        block_gemm<R, DK>(mat(Ub, 1, R), mat(bf + kC * DK, DK, 1), kC, Sr, DK, 1, 1.f, gC, stage);
     }
 }
 
 // ---------------------------------------------------------------------------
-// gdn_bwd_dscan: gradients of the chunk end states, chunks in reverse.
+// gdn_bwd_dscan: gradients of the chunk end states, chunks in reverse, with the
+// same double-buffered prefetch (diag(D) K, W, the rows of Lc, l_C).
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads) gdn_bwd_dscan(GdnBwdArgs a) {
-    constexpr int R = 16;
-    __shared__ float dS[R][DK];
-    __shared__ float X[R][kC];
-    __shared__ float stage[kKT * (kC + DK)];
+    constexpr int R = kScanRows;
+    extern __shared__ __align__(16) float dsm[];
+    float *buf[2];
+    buf[0] = dsm;
+    buf[1] = dsm + (2 * kC * DK + R * DK + 4);
+    float *dS = dsm + 2 * (2 * kC * DK + R * DK + 4);
+    float *X = dS + R * DK;
+    float *stage = X + R * kC;
     const int r0 = blockIdx.x * R, bh = blockIdx.y;
     const int nc = (a.L + kC - 1) / kC;
     const int tid = threadIdx.x;
+    // buffer layout: W [kC][DK], Kd [kC][DK], Lc rows [R][DK], l (4 floats)
+    auto prefetch = [&](int ci, float *bf) {
+        const size_t cidx = (size_t)bh * nc + ci;
+        copy_async(bf, a.bw_W + cidx * kC * DK, kC * DK);
+        copy_async(bf + kC * DK, a.bw_Kd + cidx * kC * DK, kC * DK);
+        copy_async(bf + 2 * kC * DK, a.bw_Lc + cidx * DV * DK + (size_t)r0 * DK, R * DK);
+        if (tid == 0) cp_async16(bf + 2 * kC * DK + R * DK, a.bw_ell + cidx * kC + kC - 4);
+    };
     for (int idx = tid; idx < R * DK; idx += kThreads)
-        dS[idx / DK][idx % DK] = a.dS_final ? a.dS_final[((size_t)bh * DV + r0 + idx / DK) * DK + idx % DK] : 0.f;
-    __syncthreads();
+        dS[idx] = a.dS_final ? a.dS_final[((size_t)bh * DV + r0 + idx / DK) * DK + idx % DK] : 0.f;
+    prefetch(nc - 1, buf[(nc - 1) & 1]);
+    cp_async_commit();
     for (int ci = nc - 1; ci >= 0; --ci) {
+        if (ci > 0) prefetch(ci - 1, buf[(ci - 1) & 1]);
+        cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        const float *bf = buf[ci & 1];
         const size_t cidx = (size_t)bh * nc + ci;
         float *dSg = a.bw_dS + cidx * DV * DK + (size_t)r0 * DK;
-        for (int idx = tid; idx < R * DK; idx += kThreads) dSg[idx] = dS[idx / DK][idx % DK];
+        for (int idx = tid; idx < R * DK; idx += kThreads) dSg[idx] = dS[idx];
         // X = dS_rows (diag(D) K)^T
-        block_gemm<R, kC>(mat(&dS[0][0], DK, 1), mat(a.bw_Kd + cidx * kC * DK, 1, DK), DK, &X[0][0], kC, 1, 1.f, 0.f,
-                          stage);
+        block_gemm<R, kC>(mat(dS, DK, 1), mat(bf + kC * DK, 1, DK), DK, X, kC, 1, 1.f, 0.f, stage);
         // dS_rows <- gamma_C dS_rows - X W + Lc[rows]
-        const float gC = expf(a.bw_ell[cidx * kC + kC - 1]);
-        block_gemm<R, DK>(mat(&X[0][0], kC, 1), mat(a.bw_W + cidx * kC * DK, DK, 1), kC, &dS[0][0], DK, 1, -1.f, gC,
-                          stage);
-        const float *Lc = a.bw_Lc + cidx * DV * DK + (size_t)r0 * DK;
-        for (int idx = tid; idx < R * DK; idx += kThreads) dS[idx / DK][idx % DK] += Lc[idx];
+        const float gC = expf(bf[2 * kC * DK + R * DK + 3]);
+        block_gemm<R, DK>(mat(X, kC, 1), mat(bf, DK, 1), kC, dS, DK, 1, -1.f, gC, stage);
+        for (int idx = tid; idx < R * DK; idx += kThreads) dS[idx] += bf[2 * kC * DK + idx];
         __syncthreads();
     }
     if (a.dS0)
         for (int idx = tid; idx < R * DK; idx += kThreads)
-            a.dS0[((size_t)bh * DV + r0 + idx / DK) * DK + idx % DK] = dS[idx / DK][idx % DK];
+            a.dS0[((size_t)bh * DV + r0 + idx / DK) * DK + idx % DK] = dS[idx];
 }
 
 // ---------------------------------------------------------------------------
@@ -436,9 +498,20 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_local(GdnBwdArgs a) {
 
 template <typename T, int DK, int DV>
 cudaError_t run_all(const GdnBwdArgs &a, cudaStream_t s) {
+    constexpr size_t fs = fscan_smem_floats<DK, DV>() * sizeof(float);
+    constexpr size_t ds = dscan_smem_floats<DK, DV>() * sizeof(float);
+    static_assert(fs <= 232448 && ds <= 232448, "scan shared memory exceeds 227 KB");
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(gdn_bwd_fscan<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fs);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_bwd_dscan<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ds);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
     gdn_bwd_prep<T, DK, DV><<<a.grid_chunks, kThreads, 0, s>>>(a);
-    gdn_bwd_fscan<DK, DV><<<dim3(DV / 16, a.B * a.H), kThreads, 0, s>>>(a);
-    gdn_bwd_dscan<DK, DV><<<dim3(DV / 16, a.B * a.H), kThreads, 0, s>>>(a);
+    gdn_bwd_fscan<DK, DV><<<dim3(DV / kScanRows, a.B * a.H), kThreads, fs, s>>>(a);
+    gdn_bwd_dscan<DK, DV><<<dim3(DV / kScanRows, a.B * a.H), kThreads, ds, s>>>(a);
     gdn_bwd_local<T, DK, DV><<<a.grid_chunks, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
