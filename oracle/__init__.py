@@ -18,6 +18,8 @@ Parity pins of every function: ``tests/test_oracle.py``.
 """
 from .core import (attention, attention_rows, forward, gdn, gdn_chunked, num_threads,
                    build, library_path, dswa_span, attention_backward, gdn_backward, backward)
+from .chunk_backward import gdn_backward_chunked
 
 __all__ = ["attention", "attention_rows", "forward", "gdn", "gdn_chunked", "num_threads",
-           "build", "library_path", "dswa_span", "attention_backward", "gdn_backward", "backward"]
+           "build", "library_path", "dswa_span", "attention_backward", "gdn_backward", "backward",
+           "gdn_backward_chunked"]

@@ -676,3 +676,24 @@ def test_layer_backward_gates_and_sum_match_central_differences():
     for idx in ((0, 3, 0, 1), (0, 20, 1, 3)):
         n = _central_difference(lambda a: loss_with(q=a), inp.q, idx)
         assert abs(n - g["dq"][idx]) < 1e-6 * (1 + abs(n))
+
+
+@pytest.mark.parametrize("C,L", [(64, 150), (16, 70), (64, 64)])
+def test_chunked_memory_backward_equals_recurrent_reverse_mode(C, L):
+    """The chunk form of the memory backward (the algorithm the GPU follows)
+    reproduces the token recurrence's reverse mode, including a ragged last chunk."""
+    r = np.random.default_rng(31)
+    q = rnd((1, L, 1, 8), 32)
+    k = rnd((1, L, 1, 8), 33, normalise=True)
+    v = rnd((1, L, 1, 8), 34)
+    alpha = r.uniform(0.05, 0.99, (1, L, 1)).astype(np.float32)
+    beta = r.uniform(0.05, 0.95, (1, L, 1)).astype(np.float32)
+    S0 = r.standard_normal((1, 1, 8, 8)) * 0.3
+    dSf = r.standard_normal((1, 1, 8, 8))
+    dO = r.standard_normal((1, L, 1, 8))
+    ref = oracle.gdn_backward(q, k, v, alpha, beta, dO, S0, dSf, 0)
+    f = lambda a: a[0, :, 0].astype(np.float64)
+    got = oracle.gdn_backward_chunked(f(q), f(k), f(v), f(alpha), f(beta), dO[0, :, 0], S0[0, 0], dSf[0, 0], C)
+    for name in ("dq", "dk", "dv", "dalpha", "dbeta"):
+        np.testing.assert_allclose(got[name], ref[name][0, :, 0], rtol=1e-9, atol=1e-11, err_msg=name)
+    np.testing.assert_allclose(got["dS0"], ref["dS0"][0, 0], rtol=1e-9, atol=1e-11)
