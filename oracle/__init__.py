@@ -19,6 +19,7 @@ Parity pins of every function: ``tests/test_oracle.py``.
 from .core import (attention, attention_rows, forward, gdn, gdn_chunked, num_threads,
                    build, library_path, dswa_span, attention_backward, gdn_backward, backward)
 from .chunk_backward import gdn_backward_chunked
+from . import fp8
 
 __all__ = ["attention", "attention_rows", "forward", "gdn", "gdn_chunked", "num_threads",
            "build", "library_path", "dswa_span", "attention_backward", "gdn_backward", "backward",

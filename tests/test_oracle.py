@@ -697,3 +697,44 @@ def test_chunked_memory_backward_equals_recurrent_reverse_mode(C, L):
     for name in ("dq", "dk", "dv", "dalpha", "dbeta"):
         np.testing.assert_allclose(got[name], ref[name][0, :, 0], rtol=1e-9, atol=1e-11, err_msg=name)
     np.testing.assert_allclose(got["dS0"], ref["dS0"][0, 0], rtol=1e-9, atol=1e-11)
+
+
+def test_e4m3_rounding_follows_the_format():
+    """E4M3 (4 exponent bits, bias 7, 3 mantissa bits): representable values stay,
+    ties go to the even mantissa, the subnormal spacing is 2^-9, and values past
+    the largest finite 448 saturate."""
+    r = oracle.fp8.e4m3_round
+    for x in (0.0, 1.0, 1.125, 448.0, 240.0, 2.0 ** -6, 2.0 ** -9, -3.5, 0.875):
+        assert r(x) == x
+    assert r(1.0625) == 1.0 and r(1.1875) == 1.25          # ties to even
+    assert r(3 * 2.0 ** -10) == 2.0 ** -8                  # subnormal tie to even (code 2)
+    assert r(2.0 ** -11) == 0.0 and r(2.0 ** -10 + 2.0 ** -14) == 2.0 ** -9
+    assert r(464.0) == 448.0 and r(1000.0) == 448.0 and r(-1e6) == -448.0
+    assert r(447.0) == 448.0 and r(420.0) == 416.0         # spacing 32 in [256, 448]
+
+
+def test_e4m3_rounding_matches_torch_float8():
+    """In range, the model agrees with torch's float8_e4m3fn conversion (a library
+    routine implementing the same format) on random and near-tie values."""
+    x = np.concatenate([np.random.default_rng(41).standard_normal(20000) * 30,
+                        np.random.default_rng(42).uniform(-2.0 ** -5, 2.0 ** -5, 5000)])
+    x = x[np.abs(x) <= 440].astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.fp8.e4m3_round(x), ref)
+
+
+def test_quantize_tiles_scale_and_error_bound():
+    """Per 128-row tile: the largest magnitude maps to 448 exactly, and every
+    element is within half an e4m3 spacing (relative 2^-4) of its input, or within
+    the subnormal half-spacing 2^-10 * scale."""
+    x = (np.random.default_rng(43).standard_normal((1, 300, 2, 16)) *
+         np.linspace(0.1, 10, 300)[None, :, None, None]).astype(np.float32)
+    deq, sc = oracle.fp8.quantize_tiles(x, Pseg=100)
+    assert sc.shape == (3, 2, 1)
+    for s in range(3):
+        for h in range(2):
+            tile = x[0, 100 * s:100 * (s + 1), h]
+            assert sc[s, h, 0] == np.float32(np.abs(tile).max()) / np.float32(448.0)
+            err = np.abs(deq[0, 100 * s:100 * (s + 1), h].astype(np.float64) - tile)
+            bound = np.maximum(np.abs(tile) * 2.0 ** -4, 2.0 ** -10 * sc[s, h, 0]) * (1 + 1e-6)
+            assert (err <= bound).all()

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle
-from workloads import WORKLOADS, make_inputs
+from workloads import WORKLOADS, make_inputs, bf16_to_float32
 from parity_util import (to_device, to_numpy64, run_gpu, sample_rows, oracle_rows, assert_close,
                          errors)
 
@@ -376,4 +376,25 @@ def test_fp8_logits_ragged_frames_fall_back(torch_cuda):
     out, _ = run_gpu(l8, to_device(inp))
     e = errors(to_numpy64(out), oracle.forward(inp)["out"])
     assert e["rel_l2"] <= FP8_TOL["rel_l2"] and e["max_abs"] <= FP8_TOL["max_abs"], e
+    l8.close()
+
+
+def test_fp8_logits_match_quantized_oracle(torch_cuda):
+    """The e4m3 path computes attention of the tile-quantized q and k exactly up to
+    the bf16 path's own rounding: against the oracle on the oracle's model of the
+    same quantization (codes decided in float32, as on the GPU) it meets the
+    ordinary bf16 bound."""
+    wl = WORKLOADS["clip_4k"].with_(H=4)
+    inp = make_inputs(wl, q_scale=16.0)
+    q32, k32 = bf16_to_float32(inp.q), bf16_to_float32(inp.k)
+    dev = to_device(inp)
+    g = inp.gates.astype(np.float64)
+    l8 = layer_for(wl, attn_fp8=1)
+    for i, (name, Pseg, dil, w) in enumerate((("swa", wl.L, 1, wl.swa_window),
+                                              ("dswa", wl.P, wl.dilation, wl.dswa_window))):
+        qd, _ = oracle.fp8.quantize_tiles(q32, Pseg)
+        kd, _ = oracle.fp8.quantize_tiles(k32, Pseg)
+        ref = g[None, None, :, i, None] * oracle.attention(name, qd, kd, bf16_to_float32(inp.v), wl.P, dil, w)
+        got = to_numpy64(run_gpu(l8, dev, branches=1 << i)[0])
+        assert_close(got, ref, "bf16", f"{name} fp8 vs quantized oracle")
     l8.close()
