@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-logits measurement")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="CPU time budget of the whole --impl reference run (oracle samples)")
     return ap.parse_args()
 
 
@@ -276,7 +278,7 @@ def run_reference(args, world, rank):
         return
     wl = WORKLOADS[args.workload]
     inp = make_inputs(wl)
-    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample_time(inp, per_step, seed=1)
     total, cores, desc = 0.0, 1, ""
