@@ -40,11 +40,15 @@ __device__ __forceinline__ Mat mat(const float *p, long long rs, long long cs) {
 // A(m, k) = a.at(m, k), B(k, n) = b.at(k, n); rows >= m_valid of A read as zero
 // and are not stored; beta == 0 does not read C.  stage: kKT * (M + N) floats of
 // shared memory.  Thread (tm, tn) of a 16 x 16 grid owns rows tm + 16 i and
-// columns tn + 16 j.  Begins and ends with a block barrier.
+// columns tn + 16 j.  The operands of the next kKT-deep step are loaded into
+// registers while the current step is computed.  Begins (before any operand is
+// read) and ends with a block barrier.
 template <int M, int N>
 __device__ void block_gemm(Mat a, Mat b, int K, float *c, long long crs, long long ccs, float alpha, float beta,
                            float *stage, int m_valid = M) {
     constexpr int TM = M / 16, TN = N / 16;
+    constexpr int LA = M * kKT / kThreads, LB = N * kKT / kThreads;  // staged elements per thread
+    static_assert(LA * kThreads == M * kKT && LB * kThreads == N * kKT, "tile sizes");
     float *As = stage;            // [kKT][M]
     float *Bs = stage + kKT * M;  // [kKT][N]
     const int tid = threadIdx.x, tm = tid / 16, tn = tid % 16;
@@ -53,19 +57,50 @@ __device__ void block_gemm(Mat a, Mat b, int K, float *c, long long crs, long lo
     for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
-    for (int k0 = 0; k0 < K; k0 += kKT) {
-        __syncthreads();
-        for (int idx = tid; idx < M * kKT; idx += kThreads) {
+    // staged element i of this thread: A (m, kk) and B (n, kk), laid out so that
+    // consecutive threads read along the operand's contiguous direction
+    auto a_idx = [&](int i, int &m, int &kk) {
+        const int idx = tid + i * kThreads;
+        if (a.cs == 1) { m = idx / kKT; kk = idx % kKT; } else { kk = idx / M; m = idx % M; }
+    };
+    auto b_idx = [&](int i, int &n, int &kk) {
+        const int idx = tid + i * kThreads;
+        if (b.cs == 1) { kk = idx / N; n = idx % N; } else { n = idx / kKT; kk = idx % kKT; }
+    };
+    float ra[LA], rb[LB];
+    auto load = [&](int k0) {
+#pragma unroll
+        for (int i = 0; i < LA; ++i) {
             int m, kk;
-            if (a.cs == 1) { m = idx / kKT; kk = idx % kKT; } else { kk = idx / M; m = idx % M; }
-            As[kk * M + m] = (k0 + kk < K && m < m_valid) ? a.at(m, k0 + kk) : 0.f;
+            a_idx(i, m, kk);
+            ra[i] = (k0 + kk < K && m < m_valid) ? a.at(m, k0 + kk) : 0.f;
         }
-        for (int idx = tid; idx < N * kKT; idx += kThreads) {
+#pragma unroll
+        for (int i = 0; i < LB; ++i) {
             int n, kk;
-            if (b.cs == 1) { kk = idx / N; n = idx % N; } else { n = idx / kKT; kk = idx % kKT; }
-            Bs[kk * N + n] = (k0 + kk < K) ? b.at(k0 + kk, n) : 0.f;
+            b_idx(i, n, kk);
+            rb[i] = (k0 + kk < K) ? b.at(k0 + kk, n) : 0.f;
+        }
+    };
+    // the operands may have been written by other threads just before the call
+    __syncthreads();
+    load(0);
+    for (int k0 = 0; k0 < K; k0 += kKT) {
+        if (k0 > 0) __syncthreads();  // every thread has finished reading the stage
+#pragma unroll
+        for (int i = 0; i < LA; ++i) {
+            int m, kk;
+            a_idx(i, m, kk);
+            As[kk * M + m] = ra[i];
+        }
+#pragma unroll
+        for (int i = 0; i < LB; ++i) {
+            int n, kk;
+            b_idx(i, n, kk);
+            Bs[kk * N + n] = rb[i];
         }
         __syncthreads();
+        if (k0 + kKT < K) load(k0 + kKT);
 #pragma unroll 4
         for (int kk = 0; kk < kKT; ++kk) {
             float av[TM], bv[TN];
@@ -341,7 +376,7 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_dscan(GdnBwdArgs a) {
 // gdn_bwd_local: the token gradients of one chunk per iteration.
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kThreads) gdn_bwd_local(GdnBwdArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) gdn_bwd_local(GdnBwdArgs a) {
     __shared__ ChunkScalars sc;
     __shared__ float dl[kC];
     __shared__ float red[kC][4];
