@@ -38,6 +38,8 @@
  *   - No exception crosses this boundary.  The library is not thread-safe per
  *     handle (one thread per handle at a time); distinct handles are
  *     independent.
+ *   - The calls of one handle share its device workspace: enqueue them on one
+ *     stream, or order the streams (events) so that they do not overlap.
  */
 #ifndef HLTA_H
 #define HLTA_H
